@@ -1,0 +1,336 @@
+"""Pins of the CPU oracle against facts that do not come from the oracle itself.
+
+Each test checks the oracle against one of: an independent implementation of a published algorithm
+(numpy's Philox), a distribution the draws must follow, a closed form the method reduces to
+("HyperAttention: Long-context Attention in Near-Linear Time", summary page, "Approach": with one block
+covering all keys, or with every column sampled, the estimate is exact softmax attention), an invariant
+(the estimated normaliser is at least the exact block sum; every output row is a convex combination of
+value rows), unbiasedness of the sampled normaliser, or a brute-force dense restatement of the whole
+method on tiny inputs.
+"""
+import numpy as np
+import pytest
+from scipy import stats
+
+from approximate_long_context_b200 import workload as wl
+
+
+# ---------------------------------------------------------------- independent helpers (numpy only)
+
+def exact_attention_np(Q, K, V, causal=False):
+    S = Q.astype(np.float64) @ K.astype(np.float64).T
+    if causal:
+        S = np.where(np.tril(np.ones(S.shape, bool)), S, -np.inf)
+    S = S - S.max(axis=1, keepdims=True)
+    A = np.exp(S)
+    return (A @ V.astype(np.float64)) / A.sum(axis=1, keepdims=True)
+
+
+def gray_code(k):
+    return k ^ (k >> 1)
+
+
+def ranks_np(X, P):
+    """sortLSH ranks from float64 projections: bits by sign, rank = position of the code in the
+    reflected Gray sequence (found by table lookup of the forward Gray code)."""
+    r = P.shape[1]
+    proj = X.astype(np.float64) @ P.astype(np.float64)
+    bits = (proj > 0).astype(np.int64)
+    code = (bits << np.arange(r)).sum(axis=1) if r > 0 else np.zeros(len(X), np.int64)
+    inv = np.zeros(1 << r, np.int64)
+    inv[gray_code(np.arange(1 << r))] = np.arange(1 << r)
+    return inv[code], np.abs(proj)
+
+
+def weights_noncausal(rq, rk, N, block, S):
+    """Dense weight matrix W (N x N): 1 on same-block pairs of the sorted orders, N/m on sampled columns
+    outside the query's block, 0 elsewhere."""
+    bp = min(block, N)
+    pq = np.argsort(rq, kind="stable")
+    pk = np.argsort(rk, kind="stable")
+    blk_q = np.empty(N, np.int64); blk_q[pq] = np.arange(N) // bp
+    blk_k = np.empty(N, np.int64); blk_k[pk] = np.arange(N) // bp
+    W = (blk_q[:, None] == blk_k[None, :]).astype(np.float64)
+    m = len(S)
+    if m:
+        cols = np.zeros(N, bool); cols[S] = True
+        W += np.where((blk_q[:, None] != blk_k[None, :]) & cols[None, :], N / m, 0.0)
+    return W
+
+
+def weighted_softmax_np(Q, K, V, W):
+    S = Q.astype(np.float64) @ K.astype(np.float64).T
+    S = np.where(W > 0, S, -np.inf)
+    S = S - S.max(axis=1, keepdims=True)
+    A = W * np.exp(S)
+    return (A @ V.astype(np.float64)) / A.sum(axis=1, keepdims=True), A.sum(axis=1)
+
+
+def rand_qkv(n, d, seed, planted=0.1):
+    Q, K, V = wl.make_head(n, d, seed, 0, planted, False)
+    return Q, K, V
+
+
+# ---------------------------------------------------------------- random draws
+
+@pytest.mark.parametrize("key", [(0, 0), (1234, 1), (0xDEADBEEFCAFEBABE, 2), (2**64 - 1, 2**63 + 5)])
+@pytest.mark.parametrize("ctr", [(1, 0, 0, 0), (7, 3, 2, 0), (2**40 + 3, 1, 0, 9), (5, 2**64 - 1, 2**63, 1)])
+def test_philox_matches_numpy(ora, key, ctr):
+    # numpy increments its counter before each block, so its state must hold ctr - 1 (no borrow here)
+    g = np.random.Philox(key=np.array(key, np.uint64), counter=np.array((ctr[0] - 1,) + ctr[1:], np.uint64))
+    expect = g.random_raw(4).astype(np.uint64)
+    got = ora.philox4x64_10(np.array(ctr, np.uint64), np.array(key, np.uint64))
+    assert np.array_equal(got, expect)
+
+
+def test_projection_is_standard_normal(ora):
+    vals = np.concatenate([ora.draw_projection(seed, 128, 16).ravel() for seed in range(40)])
+    assert vals.dtype == np.float32 and vals.size == 40 * 128 * 16
+    assert abs(vals.mean()) < 5 / np.sqrt(vals.size)
+    assert abs(vals.var() - 1) < 5 * np.sqrt(2 / vals.size)
+    assert stats.kstest(vals.astype(np.float64), "norm").pvalue > 1e-3
+    # deterministic in the seed, different across seeds, layout (d, r) with r columns
+    assert np.array_equal(ora.draw_projection(5, 64, 8), ora.draw_projection(5, 64, 8))
+    assert not np.array_equal(ora.draw_projection(5, 64, 8), ora.draw_projection(6, 64, 8))
+
+
+def test_projection_columns_independent(ora):
+    P = np.concatenate([ora.draw_projection(s, 64, 9) for s in range(200)], axis=0)
+    C = np.corrcoef(P.T.astype(np.float64))
+    off = C[~np.eye(9, dtype=bool)]
+    assert np.abs(off).max() < 5 / np.sqrt(P.shape[0])
+
+
+def test_samples_basic(ora):
+    for (N, m) in [(1, 1), (10, 0), (64, 64), (1000, 17), (131072, 256)]:
+        S = ora.draw_samples(99, 3, 1, N, m)
+        assert len(S) == m
+        assert np.all(np.diff(S) > 0)
+        if m:
+            assert S.min() >= 0 and S.max() < N
+    assert np.array_equal(ora.draw_samples(1, 0, 1, 50, 50), np.arange(50))
+    with pytest.raises(ValueError):
+        ora.draw_samples(1, 0, 1, 5, 6)
+    a, b, c = ora.draw_samples(1, 0, 1, 1000, 20), ora.draw_samples(1, 1, 1, 1000, 20), ora.draw_samples(1, 0, 2, 1000, 20)
+    assert not np.array_equal(a, b) and not np.array_equal(a, c)
+
+
+def test_samples_uniform(ora):
+    N, m, T = 64, 8, 4000
+    counts = np.zeros(N)
+    pair = np.zeros((N, N))
+    for seed in range(T):
+        S = ora.draw_samples(seed, 0, 1, N, m)
+        counts[S] += 1
+        pair[np.ix_(S, S)] += 1
+    exp = T * m / N
+    chi2 = ((counts - exp) ** 2 / exp).sum()
+    assert stats.chi2.sf(chi2, N - 1) > 1e-4
+    # pairwise inclusion probability m(m-1)/(N(N-1)) for every pair (without replacement)
+    p2 = pair[~np.eye(N, dtype=bool)] / T
+    target = m * (m - 1) / (N * (N - 1))
+    assert abs(p2.mean() - target) < 1e-3
+
+
+# ---------------------------------------------------------------- hash
+
+def test_gray_rank_inverse_and_adjacency(ora):
+    for k in range(1 << 16):
+        assert ora.gray_rank(gray_code(k)) == k
+    for k in range((1 << 16) - 1):
+        assert bin(gray_code(k) ^ gray_code(k + 1)).count("1") == 1
+
+
+@pytest.mark.parametrize("d,r", [(64, 6), (64, 8), (128, 7), (128, 9), (32, 16), (64, 0)])
+def test_hash_matches_float64_signs(ora, d, r):
+    X = np.random.default_rng(d * 100 + r).standard_normal((4000, d)).astype(np.float32) * np.float32(d ** -0.25)
+    P = ora.draw_projection(77, d, r)
+    rank, near = ora.hash_rows(X, P)
+    ref, absproj = ranks_np(X, P)
+    norms = np.linalg.norm(X.astype(np.float64), axis=1)
+    # a projection far from zero decides its bit identically in fp32 and float64
+    safe = (absproj >= 1e-3 * norms[:, None]).all(axis=1) if r else np.ones(len(X), bool)
+    assert safe.mean() > 0.9
+    assert np.array_equal(rank[safe].astype(np.int64), ref[safe])
+    # the near-zero flag marks exactly the rows with a projection below 1e-4 * ||x|| (up to fp32 rounding)
+    clearly_near = (absproj < 0.9e-4 * norms[:, None]).any(axis=1) if r else np.zeros(len(X), bool)
+    clearly_far = (absproj > 1.1e-4 * norms[:, None]).all(axis=1) if r else np.ones(len(X), bool)
+    assert near[clearly_near].all() and not near[clearly_far].any()
+    if r == 0:
+        assert (rank == 0).all()
+
+
+def test_hash_sign_tie_is_zero_bit(ora):
+    X = np.zeros((3, 16), np.float32)
+    X[1, 0] = 1.0
+    X[2, 0] = X[2, 1] = 1.0
+    P = np.ones((16, 4), np.float32)
+    P[0, 1] = -1.0
+    P[1, 2] = -1.0
+    rank, near = ora.hash_rows(X, P)
+    # zero row: every projection is exactly 0 -> code 0; |p| < 1e-4 * 0 is false, so it is not flagged
+    assert rank[0] == 0 and near[0] == 0
+    # e_0: projections (1, -1, 1, 1) -> code 0b1101
+    assert rank[1] == ora.gray_rank(0b1101) and near[1] == 0
+    # e_0 + e_1: projections (2, 0, 0, 2) -> exact zeros give bit 0 and flag the row
+    assert rank[2] == ora.gray_rank(0b1001) and near[2] == 1
+
+
+def test_sort_stable(ora):
+    rng = np.random.default_rng(3)
+    for R in [1, 4, 256, 65536]:
+        rank = rng.integers(0, R, 5000).astype(np.uint16)
+        assert np.array_equal(ora.sort_segment(rank), np.argsort(rank, kind="stable"))
+
+
+# ---------------------------------------------------------------- closed forms and invariants
+
+@pytest.mark.parametrize("n,d,m,r", [(256, 32, 16, 4), (512, 64, 0, 6), (128, 16, 128, 3)])
+def test_block_n_equals_exact(ora, n, d, m, r):
+    Q, K, V = rand_qkv(n, d, 11)
+    out = ora.forward(Q, K, V, block=n, m=m, r=r, causal=False, seed=5)
+    np.testing.assert_allclose(out["O"], exact_attention_np(Q, K, V), rtol=1e-10, atol=1e-12)
+    # the oracle's own exact routine agrees with the textbook formula too
+    np.testing.assert_allclose(ora.exact_attention(Q, K, V, causal=False), exact_attention_np(Q, K, V), rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("n,block,r", [(256, 16, 5), (512, 64, 6), (128, 128, 2)])
+def test_all_columns_sampled_equals_exact(ora, n, block, r):
+    Q, K, V = rand_qkv(n, 32, 12)
+    out = ora.forward(Q, K, V, block=block, m=n, r=r, causal=False, seed=6)
+    np.testing.assert_allclose(out["O"], exact_attention_np(Q, K, V), rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("n,block", [(256, 16), (1024, 64), (192, 64)])
+def test_no_samples_identical_codes_is_block_diagonal(ora, n, block):
+    Q, K, V = rand_qkv(n, 32, 13)
+    out = ora.forward(Q, K, V, block=block, m=0, r=0, causal=False, seed=7)
+    ref = np.concatenate([exact_attention_np(Q[i:i + block], K[i:i + block], V[i:i + block])
+                          for i in range(0, n, block)])
+    np.testing.assert_allclose(out["O"], ref, rtol=1e-10, atol=1e-12)
+
+
+def test_normaliser_at_least_block_sum(ora):
+    Q, K, V = rand_qkv(1024, 64, 14)
+    out = ora.forward(Q, K, V, block=64, m=64, r=6, causal=False, seed=8, want_parts=True)
+    L, L1, L2 = out["L"], out["L1"], out["L2"]
+    assert np.all(L >= L1)
+    np.testing.assert_allclose(L, np.logaddexp(L1, L2), rtol=0, atol=1e-12)
+    assert np.isfinite(L2).mean() > 0.99
+
+
+def test_normaliser_unbiased(ora):
+    n, d, block, m, r, T = 64, 16, 8, 8, 3, 10000
+    Q, K, V = rand_qkv(n, d, 15, planted=0.2)
+    D = np.exp(Q.astype(np.float64) @ K.astype(np.float64).T).sum(axis=1)
+    est = np.zeros((T, n))
+    for seed in range(T):
+        est[seed] = np.exp(ora.forward(Q, K, V, block=block, m=m, r=r, causal=False, seed=seed)["L"])
+    mean = est.mean(axis=0)
+    se = est.std(axis=0, ddof=1) / np.sqrt(T)
+    z = (mean - D) / se
+    assert np.abs(z).max() < 5.0, np.abs(z).max()
+
+
+def test_rows_are_convex_combinations(ora):
+    Q, K, V = rand_qkv(2048, 64, 16)
+    lo, hi = V.min(axis=0).astype(np.float64), V.max(axis=0).astype(np.float64)
+    for causal, base in [(False, 0), (True, 256)]:
+        O = ora.forward(Q, K, V, block=64, m=32, r=6, causal=causal, base=base, seed=9)["O"]
+        assert np.all(O >= lo - 1e-12) and np.all(O <= hi + 1e-12)
+
+
+# ---------------------------------------------------------------- causal
+
+def test_causal_base_at_least_n_is_exact_causal(ora):
+    Q, K, V = rand_qkv(300, 32, 17)
+    out = ora.forward(Q, K, V, block=50, m=10, r=5, causal=True, base=300, seed=10)
+    np.testing.assert_allclose(out["O"], exact_attention_np(Q, K, V, causal=True), rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("n,base,m", [(256, 32, 0), (256, 32, 32), (512, 64, 17)])
+def test_causal_full_blocks_are_exact_causal(ora, n, base, m):
+    Q, K, V = rand_qkv(n, 32, 18)
+    out = ora.forward(Q, K, V, block=n, m=m, r=6, causal=True, base=base, seed=11)
+    np.testing.assert_allclose(out["O"], exact_attention_np(Q, K, V, causal=True), rtol=1e-10, atol=1e-12)
+
+
+def test_causal_rejects_bad_shapes(ora):
+    Q, K, V = rand_qkv(96, 16, 19)
+    with pytest.raises(ValueError):
+        ora.forward(Q, K, V, block=16, m=4, r=3, causal=True, base=64, seed=1)   # 96 != 64 * 2^L
+    Q, K, V = rand_qkv(128, 16, 19)
+    with pytest.raises(ValueError):
+        ora.forward(Q, K, V, block=16, m=40, r=3, causal=True, base=32, seed=1)  # m > smallest N = 32
+
+
+# ---------------------------------------------------------------- dense brute force of the whole method
+
+def _dense_causal_weights(Q, K, P, block, base, m, seed, bh, ora):
+    n = len(Q)
+    rq_all, aq = ranks_np(Q, P)
+    rk_all, ak = ranks_np(K, P)
+    W = np.zeros((n, n))
+    leaf = min(base, n)
+    for q in range(n):
+        lo = q - q % leaf
+        W[q, lo:q + 1] = 1.0
+
+    def rec(node, s, length):
+        if length <= leaf:
+            return
+        h = length // 2
+        rec(2 * node, s, h)
+        rec(2 * node + 1, s + h, h)
+        S = ora.draw_samples(seed, bh, node, h, m)
+        W[s + h:s + length, s:s + h] = weights_noncausal(rq_all[s + h:s + length], rk_all[s:s + h], h, block, S)
+
+    rec(1, 0, n)
+    return W, np.concatenate([aq, ak])
+
+
+@pytest.mark.parametrize("seed", [21, 22, 23])
+@pytest.mark.parametrize("causal", [False, True])
+def test_dense_bruteforce(ora, seed, causal):
+    n, d, block, m, r, base, bh = 256, 16, 16, 12, 4, 32, 3
+    Q, K, V = rand_qkv(n, d, seed)
+    P = ora.draw_projection(seed, d, r)
+    if causal:
+        W, absproj = _dense_causal_weights(Q, K, P, block, base, m, seed, bh, ora)
+    else:
+        rq, aq = ranks_np(Q, P)
+        rk, ak = ranks_np(K, P)
+        W = weights_noncausal(rq, rk, n, block, ora.draw_samples(seed, bh, 1, n, m))
+        absproj = np.concatenate([aq, ak])
+    X = np.concatenate([Q, K]).astype(np.float64)
+    # fp32 and float64 take the same sign decisions when no projection is within 1e-5 * ||x|| of zero
+    assert (absproj >= 1e-5 * np.linalg.norm(X, axis=1)[:, None]).all(), "pick a seed without near-zero projections"
+    ref, den = weighted_softmax_np(Q, K, V, W)
+    out = ora.forward(Q, K, V, block=block, m=m, r=r, causal=causal, base=base, seed=seed, bh=bh)
+    np.testing.assert_allclose(out["O"], ref, rtol=1e-10, atol=1e-12)
+    S = Q.astype(np.float64) @ K.astype(np.float64).T
+    mx = np.where(W > 0, S, -np.inf).max(axis=1)
+    np.testing.assert_allclose(out["L"], mx + np.log(den), rtol=0, atol=1e-10)
+
+
+def test_rows_subset_matches_full(ora):
+    Q, K, V = rand_qkv(1024, 32, 24)
+    rows = np.array([0, 5, 511, 512, 777, 1023])
+    for causal in (False, True):
+        full = ora.forward(Q, K, V, block=32, m=16, r=5, causal=causal, base=128, seed=3)
+        part = ora.forward(Q, K, V, block=32, m=16, r=5, causal=causal, base=128, seed=3, rows=rows)
+        np.testing.assert_array_equal(part["O"], full["O"][rows])
+
+
+def test_level_perms(ora):
+    rng = np.random.default_rng(5)
+    n = 512
+    rank = rng.integers(0, 16, 2 * n).astype(np.uint16)
+    pq, pk = ora.level_perms(rank, n, 0)
+    assert np.array_equal(pq, np.argsort(rank[:n], kind="stable"))
+    assert np.array_equal(pk, np.argsort(rank[n:], kind="stable"))
+    pq, pk = ora.level_perms(rank, n, 2)            # nodes of length 256: Q lower / K upper halves of 128
+    for j in range(2):
+        s = j * 256
+        assert np.array_equal(pq[j * 128:(j + 1) * 128], np.argsort(rank[s + 128:s + 256], kind="stable"))
+        assert np.array_equal(pk[j * 128:(j + 1) * 128], np.argsort(rank[n + s:n + s + 128], kind="stable"))

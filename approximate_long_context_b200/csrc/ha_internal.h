@@ -1,0 +1,73 @@
+// ha_internal.h -- declarations shared by the library's translation units (not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ha {
+
+constexpr int kMaxR = 16;            // hash bits
+constexpr int kMaxPassBits = 10;     // radix digit of one counting-sort pass (<= 1024 buckets)
+constexpr int kSortChunk = 2048;     // rows per counting-sort chunk (one CTA)
+constexpr int kSortWarps = 8;
+
+// Device status word bits (written by kernels that wait with a bound, read by hyper_attn_status).
+constexpr int kStatusTimeout = 1;
+
+// One level of the computation. Level 0 is the non-causal problem (one node covering all n rows);
+// causal level l >= 1 has nodes of node_len = n >> (l-1) rows whose off-diagonal problem pairs the
+// query rows [q_off, node_len) with the key rows [0, seg_len) of the node (q_off = seg_len = node_len/2).
+struct Level {
+    int64_t n;          // rows per (batch, head)
+    int64_t bh;         // batch * heads
+    int64_t nodes;      // nodes at this level
+    int64_t node_len;   // rows per node
+    int64_t seg_len;    // N: query rows = key rows of one problem
+    int64_t q_off;      // first query row of a node, relative to the node start
+    int64_t heap0;      // heap id of node 0 of this level
+    int level;          // 0 = non-causal, >= 1 causal level
+    int bp;             // block size b' = min(block, N)
+};
+
+// Sort pass description: digit = (rank >> shift) & (radix - 1).
+struct SortPass {
+    int shift;
+    int radix;          // power of two <= 1 << kMaxPassBits
+};
+
+// ---- kernels (launch wrappers return the number of kernels launched, or -1 on launch error) ----
+
+// sortLSH hash of 2*bh*n rows (Q rows then K rows of each problem): rank[bh][2][n], near[bh][2][n].
+int launch_hash(const void *Q, const void *K, int dtype, int64_t bh, int64_t n, int d, const float *P, int r,
+                uint16_t *rank, uint8_t *near, cudaStream_t st);
+
+// Stable counting sort of all segments of a level by one digit.
+//   in_idx: nullptr (rows in natural order) or the previous pass's permutation (same layout as perm).
+//   perm[s*N + pos] = local row; inv[s*N + row] = pos (inv may be nullptr).
+int launch_sort_pass(const Level &lv, const uint16_t *rank, SortPass ps, const int32_t *in_idx,
+                     int32_t *hist, int32_t *perm, int32_t *inv, cudaStream_t st);
+
+// SIMT attention of one level: for level 0 writes O (out dtype); for causal levels writes the parts
+// Opart[bh][n/2][d] (fp32, normalised) and Lpart[bh][n/2] (log normaliser) of this level.
+int launch_attn_simt(const Level &lv, const void *Q, const void *K, const void *V, int dtype, int d,
+                     const int32_t *perm, const int32_t *inv, const int32_t *S, int m, int64_t nodes_total,
+                     void *O, int out_dtype, float *lse, float *Opart, float *Lpart, cudaStream_t st);
+
+// SIMT exact causal attention on leaves of `leaf` rows, merged with the parts of levels 1..L.
+int launch_causal_base_simt(const void *Q, const void *K, const void *V, int dtype, int64_t bh, int64_t n,
+                            int d, int64_t leaf, int levels, const float *Opart, const float *Lpart,
+                            void *O, int out_dtype, cudaStream_t st);
+
+// Tensor-core (tcgen05) kernels; return -2 when a shape is not supported by the tensor-core path.
+int launch_attn_tc(const Level &lv, const void *Q, const void *K, const void *V, int d,
+                   const int32_t *perm, const int32_t *inv, const int32_t *S, int m, int64_t nodes_total,
+                   void *O, int out_dtype, float *lse, float *Opart, float *Lpart, int *status, cudaStream_t st);
+int launch_causal_base_tc(const void *Q, const void *K, const void *V, int64_t bh, int64_t n, int d,
+                          int64_t leaf, int levels, const float *Opart, const float *Lpart,
+                          void *O, int out_dtype, int *status, cudaStream_t st);
+
+// ---- host-side draws (ha_draws.cpp) ----
+void draw_projection(uint64_t seed, int d, int r, float *P);
+int draw_samples(uint64_t seed, uint64_t bh, uint64_t node, int64_t N, int m, int32_t *S, uint8_t *scratch);
+
+}  // namespace ha

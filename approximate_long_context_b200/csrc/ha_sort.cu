@@ -1,0 +1,167 @@
+// ha_sort.cu -- stable segmented counting sort of the sortLSH ranks.
+//
+// "HyperAttention: Long-context Attention in Near-Linear Time" (research-map summary, "Approach"): the
+// rows of Q and of K are sorted by their LSH bucket rank. Ties keep the original row order (stable), so the
+// sorted order is unique. Every problem of a level has one query segment and one key segment of N rows
+// (see ha::Level); segment s = (bh * nodes + node) * 2 + which, which 0 = queries, 1 = keys.
+//
+// One pass sorts by one radix digit of at most 10 bits; ranks of up to 16 bits take two stable passes
+// (least significant digit first). A pass is three launches:
+//   count   -- per 2048-row chunk of a segment, a shared-memory histogram of the digit;
+//   scan    -- per segment, turn the chunk histograms into the first output position of every
+//              (chunk, digit) pair (digit-major, chunks in order);
+//   scatter -- per chunk, 8 warps each own a contiguous 256-row slice; a warp ranks equal digits inside a
+//              32-row step with __match_any_sync and keeps running per-digit counters, so rows leave in
+//              their original order within each digit.
+// No kernel waits on another CTA: the three launches replace a look-back scan.
+#include "ha_common.cuh"
+#include "ha_internal.h"
+
+namespace ha {
+namespace {
+
+struct SegView {
+    const uint16_t *rank;   // rank of local row 0 of the segment
+    int64_t out;            // s * N: first slot of the segment in perm / inv
+};
+
+__device__ __forceinline__ SegView seg_view(const Level &lv, const uint16_t *rank, int64_t s) {
+    const int64_t which = s & 1;
+    const int64_t node = (s >> 1) % lv.nodes;
+    const int64_t bhi = (s >> 1) / lv.nodes;
+    const int64_t start = node * lv.node_len + (which == 0 ? lv.q_off : 0);
+    SegView v;
+    v.rank = rank + (bhi * 2 + which) * lv.n + start;
+    v.out = s * lv.seg_len;
+    return v;
+}
+
+__device__ __forceinline__ int digit_of(const SegView &v, const int32_t *in_idx, int64_t p, SortPass ps,
+                                        int32_t &row) {
+    row = in_idx ? in_idx[v.out + p] : static_cast<int32_t>(p);
+    return (static_cast<int>(v.rank[row]) >> ps.shift) & (ps.radix - 1);
+}
+
+__global__ void __launch_bounds__(256) sort_count_kernel(Level lv, const uint16_t *__restrict__ rank, SortPass ps,
+                                                         const int32_t *__restrict__ in_idx, int32_t *__restrict__ hist,
+                                                         int cps) {
+    extern __shared__ int cnt[];
+    const int64_t s = blockIdx.x / cps;
+    const int c = blockIdx.x % cps;
+    for (int b = threadIdx.x; b < ps.radix; b += blockDim.x) cnt[b] = 0;
+    __syncthreads();
+    const SegView v = seg_view(lv, rank, s);
+    const int64_t start = static_cast<int64_t>(c) * kSortChunk;
+    const int64_t end = min(lv.seg_len, start + kSortChunk);
+    for (int64_t p = start + threadIdx.x; p < end; p += blockDim.x) {
+        int32_t row;
+        atomicAdd(&cnt[digit_of(v, in_idx, p, ps, row)], 1);
+    }
+    __syncthreads();
+    int32_t *h = hist + (s * cps + c) * ps.radix;
+    for (int b = threadIdx.x; b < ps.radix; b += blockDim.x) h[b] = cnt[b];
+}
+
+__global__ void __launch_bounds__(1024) sort_scan_kernel(int radix, int cps, int32_t *__restrict__ hist) {
+    __shared__ int tot[1 << kMaxPassBits];
+    const int64_t s = blockIdx.x;
+    int32_t *h = hist + s * cps * radix;
+    for (int b = threadIdx.x; b < radix; b += blockDim.x) {
+        int run = 0;
+        for (int c = 0; c < cps; ++c) {
+            const int t = h[c * radix + b];
+            h[c * radix + b] = run;
+            run += t;
+        }
+        tot[b] = run;
+    }
+    __syncthreads();
+    // inclusive scan of the digit totals (Hillis-Steele; radix <= blockDim, one digit per thread)
+    const int b = threadIdx.x;
+    for (int off = 1; off < radix; off <<= 1) {
+        const int add = (b < radix && b >= off) ? tot[b - off] : 0;
+        __syncthreads();
+        if (b < radix) tot[b] += add;
+        __syncthreads();
+    }
+    if (b < radix) {
+        const int base = b == 0 ? 0 : tot[b - 1];
+        for (int c = 0; c < cps; ++c) h[c * radix + b] += base;
+    }
+}
+
+__global__ void __launch_bounds__(kSortWarps * 32) sort_scatter_kernel(Level lv, const uint16_t *__restrict__ rank,
+                                                                       SortPass ps, const int32_t *__restrict__ in_idx,
+                                                                       const int32_t *__restrict__ hist, int cps,
+                                                                       int32_t *__restrict__ perm,
+                                                                       int32_t *__restrict__ inv) {
+    extern __shared__ int wcnt[];   // [kSortWarps][radix]
+    const int64_t s = blockIdx.x / cps;
+    const int c = blockIdx.x % cps;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (int i = threadIdx.x; i < kSortWarps * ps.radix; i += blockDim.x) wcnt[i] = 0;
+    __syncthreads();
+
+    const SegView v = seg_view(lv, rank, s);
+    const int64_t start = static_cast<int64_t>(c) * kSortChunk;
+    const int64_t end = min(lv.seg_len, start + kSortChunk);
+    constexpr int kSlice = kSortChunk / kSortWarps;
+    const int64_t lo = min(end, start + static_cast<int64_t>(warp) * kSlice);
+    const int64_t hi = min(end, lo + kSlice);
+    int *mycnt = wcnt + warp * ps.radix;
+
+    for (int64_t base = lo; base < hi; base += 32) {
+        const int64_t p = base + lane;
+        const bool valid = p < hi;
+        int32_t row = 0;
+        const int key = valid ? digit_of(v, in_idx, p, ps, row) : -1;
+        const unsigned peers = __match_any_sync(0xffffffffu, key);
+        if (valid && lane == __ffs(peers) - 1) mycnt[key] += __popc(peers);
+    }
+    __syncthreads();
+    const int32_t *h = hist + (s * cps + c) * ps.radix;
+    for (int b = threadIdx.x; b < ps.radix; b += blockDim.x) {
+        int run = h[b];
+        for (int w = 0; w < kSortWarps; ++w) {
+            const int t = wcnt[w * ps.radix + b];
+            wcnt[w * ps.radix + b] = run;
+            run += t;
+        }
+    }
+    __syncthreads();
+    for (int64_t base = lo; base < hi; base += 32) {
+        const int64_t p = base + lane;
+        const bool valid = p < hi;
+        int32_t row = 0;
+        const int key = valid ? digit_of(v, in_idx, p, ps, row) : -1;
+        const unsigned peers = __match_any_sync(0xffffffffu, key);
+        const int first = valid ? mycnt[key] : 0;
+        __syncwarp();
+        if (valid && lane == __ffs(peers) - 1) mycnt[key] = first + __popc(peers);
+        __syncwarp();
+        if (valid) {
+            const int pos = first + __popc(peers & lt_mask);
+            perm[v.out + pos] = row;
+            if (inv) inv[v.out + row] = pos;
+        }
+    }
+}
+
+}  // namespace
+
+int launch_sort_pass(const Level &lv, const uint16_t *rank, SortPass ps, const int32_t *in_idx, int32_t *hist,
+                     int32_t *perm, int32_t *inv, cudaStream_t st) {
+    if (ps.radix < 1 || ps.radix > (1 << kMaxPassBits)) return -1;
+    const int64_t nseg = lv.bh * lv.nodes * 2;
+    const int cps = static_cast<int>((lv.seg_len + kSortChunk - 1) / kSortChunk);
+    const int64_t grid = nseg * cps;
+    sort_count_kernel<<<static_cast<unsigned>(grid), 256, ps.radix * sizeof(int), st>>>(lv, rank, ps, in_idx, hist, cps);
+    sort_scan_kernel<<<static_cast<unsigned>(nseg), 1024, 0, st>>>(ps.radix, cps, hist);
+    const size_t smem = static_cast<size_t>(kSortWarps) * ps.radix * sizeof(int);
+    sort_scatter_kernel<<<static_cast<unsigned>(grid), kSortWarps * 32, smem, st>>>(lv, rank, ps, in_idx, hist, cps,
+                                                                                    perm, inv);
+    return cudaPeekAtLastError() == cudaSuccess ? 3 : -1;
+}
+
+}  // namespace ha

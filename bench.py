@@ -1,0 +1,374 @@
+#!/usr/bin/env python
+"""Benchmark of the HyperAttention forward pass (one JSON line on rank 0).
+
+Metric: forward throughput in Mqueries*heads/s (batch * heads * n / time) on the n = 131072 single-layer
+workload (32 heads, d = 64, block 256, m = 256, r = 8, bf16), with the achieved fraction of the roofline of
+the dominant kernel class. A step is one full forward pass (hash, sort, attention with gather and merge)
+over the resident inputs. Multi-GPU runs are weak scaling: every rank runs its own full workload (the
+problems are independent, no collective on the data path); value = all ranks' queries*heads / max time.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from approximate_long_context_b200 import workload as wl  # noqa: E402
+
+L2_BYTES = 126 * 2 ** 20
+FP32_SIMT_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # SMs x FP32 lanes x 2 flop/FMA x max SM clock
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM bytes per launch of a kernel class from an ncu capture, valid only while the source file it was
+# taken from is unchanged (sha256 of the file at capture time).
+TRAFFIC = {}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"])}, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def algorithmic(w: wl.Workload, cls: str):
+    """Algorithmic work per launch of a kernel class: (bytes, flops)."""
+    e = 2 if w.dtype == "bf16" else 4
+    bh, n, d = w.bh, w.n, w.d
+    levels = 0
+    if w.causal and w.n > w.base:
+        levels = int(round(np.log2(w.n // w.base)))
+    if cls == "hash":
+        return bh * 2 * n * (d * e + 3), 0.0                    # read Q, K rows; write rank (2 B) + flag (1 B)
+    if cls == "sort":
+        rows = bh * 2 * n if not w.causal else bh * n            # rows sorted per level
+        return rows * (2 + 2 + 4 + 4), 0.0                       # rank read twice, perm + inverse written
+    if cls == "attn":
+        N = n if not w.causal else n // 2                        # query rows per level launch
+        flops = bh * 4.0 * N * d * (min(w.block, N if not w.causal else n) + w.m)
+        byts = bh * N * (3 * d * e + d * (e if not w.causal else 4) + 8)
+        return byts, flops
+    if cls == "causal_base":
+        flops = bh * 2.0 * n * d * w.base
+        byts = bh * n * (3 * d * e + d * e) + bh * n * levels * (d * 4 + 4) / 2
+        return byts, flops
+    raise KeyError(cls)
+
+
+class ClockSampler:
+    """Samples SM clock, power and clock-event reasons of one GPU with NVML while running."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, torch_device_index: int, period_s: float = 0.02):
+        self.samples = []
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thr = None
+        self.handle = None
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            import torch
+            props = torch.cuda.get_device_properties(torch_device_index)
+            bus = getattr(props, "pci_bus_id", None)
+            dom = getattr(props, "pci_domain_id", 0)
+            dev = getattr(props, "pci_device_id", 0)
+            if bus is not None:
+                busid = f"{dom:08X}:{bus:02X}:{dev:02X}.0"
+                self.handle = pynvml.nvmlDeviceGetHandleByPciBusId(busid)
+            else:
+                self.handle = pynvml.nvmlDeviceGetHandleByIndex(torch_device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+        except Exception as exc:  # clocks are reported as unavailable rather than guessed
+            self.error = str(exc)
+            self.handle = None
+
+    def _run(self):
+        nv = self.nvml
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                self.samples.append((sm, reasons))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.handle is not None:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._thr:
+            self._thr.join()
+
+    def summary(self):
+        if self.handle is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "note": "NVML unavailable: " + getattr(self, "error", "")}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        sms = [s for s, _ in self.samples]
+        reasons = set()
+        for _, r in self.samples:
+            for bit, name in self.REASONS.items():
+                if r & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons),
+                "samples": len(sms)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def cpu_oracle_rate(w: wl.Workload, heads):
+    """Oracle time on full heads (all rows): returns (Mqueries*heads/s, seconds, threads)."""
+    import oracle
+    oracle.build()
+    Qh, Kh, Vh = wl.workload_inputs(w, heads=heads)
+    t0 = time.perf_counter()
+    for i, h in enumerate(heads):
+        oracle.forward(wl.as_f32(Qh[i]), wl.as_f32(Kh[i]), wl.as_f32(Vh[i]), block=w.block, m=w.m, r=w.r,
+                       causal=w.causal, base=w.base, seed=w.algo_seed, bh=h)
+    dt = time.perf_counter() - t0
+    return len(heads) * w.n / dt / 1e6, dt, oracle.num_threads()
+
+
+def run_reference(args, w: wl.Workload):
+    world, rank, _ = dist_setup()
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    head = [0]
+    Qh, Kh, Vh = wl.workload_inputs(w, heads=head)
+    Qf, Kf, Vf = wl.as_f32(Qh[0]), wl.as_f32(Kh[0]), wl.as_f32(Vh[0])
+
+    def step():
+        oracle.forward(Qf, Kf, Vf, block=w.block, m=w.m, r=w.r, causal=w.causal, base=w.base, seed=w.algo_seed, bh=0)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    value = w.n / dt / 1e6
+    sample = f"1 of {w.bh} heads per step, all {w.n} query rows (hash, sort and attention of that head)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+METRIC = "HyperAttention fwd Mqueries\u00b7heads/s at n=131k; % of BF16 tensor/HBM roofline"
+UNIT = "Mqueries\u00b7heads/s"
+
+
+def config_of(w: wl.Workload):
+    return {"workload": w.name, "batch": w.batch, "heads": w.heads, "n": w.n, "d": w.d, "block": w.block, "m": w.m,
+            "r": w.r, "causal": w.causal, "causal_base": w.base if w.causal else None, "input_dtype": w.dtype,
+            "parallelism": "independent (batch, head) problems per GPU; no collective",
+            "l2": "inputs larger than L2, no flush" if 3 * w.bh * w.n * w.d * 2 > 2 * L2_BYTES else "L2 flushed"}
+
+
+def run_ours(args, w: wl.Workload):
+    import torch
+    import torch.distributed as dist
+    from approximate_long_context_b200 import binding
+
+    world, rank, local = dist_setup()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    esz = 2 if w.dtype == "bf16" else 4
+    Qh, Kh, Vh = wl.workload_inputs(w)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+    def pinned(a):
+        t = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a)
+        p = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        p.copy_(t)
+        return p.view(tdt) if w.dtype == "bf16" else p
+
+    hQ, hK, hV = pinned(Qh), pinned(Kh), pinned(Vh)
+    del Qh, Kh, Vh
+    hO = torch.empty(hQ.shape, dtype=tdt, pin_memory=True)
+    Q, K, V = hQ.to(dev), hK.to(dev), hV.to(dev)
+    O = torch.empty_like(Q)
+    stream = torch.cuda.current_stream(dev)
+    flush = None if 3 * Q.numel() * esz > 2 * L2_BYTES else torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+
+    ha = binding.HyperAttention(local)
+    ha.set_options(dtype=w.dtype, batch=w.batch, causal_base=w.base or 4096, stream=stream.cuda_stream,
+                   kernel=args.kernel)
+    kw = dict(n=w.n, d=w.d, heads=w.heads, block=w.block, m=w.m, r=w.r, causal=w.causal, seed=w.algo_seed)
+
+    def step():
+        if flush is not None:
+            flush.zero_()
+        ha.forward(Q, K, V, O, **kw)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    launches_per_step = ha.last_launch_count()
+    ha.profile_read()          # drop anything recorded during warm-up
+    ha.profile(True)
+
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier()
+    ha.profile(False)
+    prof = ha.profile_read()
+    assert ha.status() == 0, ha.last_error()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    t = torch.tensor([ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    units = world * w.bh * w.n
+    value = units / (ms_max * 1e-3) / 1e6
+
+    # end to end through the host-buffer entry point: H2D of Q, K, V and D2H of O inside the timed region
+    for _ in range(1):
+        ha.forward_host(hQ, hK, hV, hO, **kw)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(args.steps):
+        ha.forward_host(hQ, hK, hV, hO, **kw)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    te = torch.tensor([e0.elapsed_time(e1) / args.steps], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_value = units / (float(te.item()) * 1e-3) / 1e6
+
+    # roofline of the dominant kernel class; sort and attention launch once per level
+    peaks, peak_src = load_peaks()
+    family = ha.last_kernel()
+    dom = max(prof, key=lambda k: prof[k][0])
+    dom_ms = prof[dom][0]
+    nlev = int(round(np.log2(w.n // w.base))) if (w.causal and w.n > w.base) else (0 if w.causal else 1)
+    groups = nlev if dom in ("sort", "attn") else 1
+    avg_ms = dom_ms / (args.steps * groups)
+    byts, flops = algorithmic(w, dom)
+    if flops > 0 and dom in ("attn", "causal_base"):
+        if family == "tc":
+            bound, peak, unit = "tensor", peaks["bf16_tflops"], "TFLOP/s"
+        else:
+            bound, peak, unit = "alu", FP32_SIMT_PEAK_TFLOPS, "TFLOP/s"
+        achieved = flops / (avg_ms * 1e-3) / 1e12
+    else:
+        bound, peak, unit = "hbm", peaks["hbm_gbs"], "GB/s"
+        achieved = byts / (avg_ms * 1e-3) / 1e9
+    traffic = None
+    tr = TRAFFIC.get((dom, w.name, family))
+    if tr is not None:
+        src = os.path.join(ROOT, "approximate_long_context_b200", "csrc", tr["file"])
+        if os.path.exists(src) and hashlib.sha256(open(src, "rb").read()).hexdigest() == tr["sha256"]:
+            traffic = tr["bytes"]
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        heads = list(range(min(args.cpu_heads, w.bh)))
+        rate, secs, cores = cpu_oracle_rate(w, heads)
+        cpu = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"{len(heads)} of {w.bh} heads, all {w.n} query rows ({secs:.1f} s)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded Gaussian Q/K/V, planted heavy keys)",
+            "config": config_of(w),
+            "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                         "frac": achieved / peak, "traffic": traffic, "kernel": dom,
+                         "kernel_ms_per_launch": avg_ms, "peak_source": peak_src + (" burst" if bound == "tensor" else ""),
+                         "kernel_family": "tcgen05" if family == "tc" else "simt"},
+            "kernel_ms_per_step": {k: v[0] / args.steps for k, v in prof.items()},
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": 3 * Q.numel() * esz,
+                    "d2h_bytes_per_step": O.numel() * esz},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk.summary(),
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    ha.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=wl.HEADLINE, choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--kernel", default="auto", choices=["auto", "simt", "tc"])
+    ap.add_argument("--cpu-heads", type=int, default=4)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    w = wl.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

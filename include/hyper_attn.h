@@ -1,0 +1,174 @@
+/*
+ * hyper_attn.h -- C ABI of the B200-native HyperAttention forward pass (sm_100a).
+ *
+ * The method ("HyperAttention: Long-context Attention in Near-Linear Time"; research-map summary page,
+ * section "Approach", and the OpenReview abstract): hash the rows of Q and K with sortLSH (signs of r
+ * random Gaussian projections read as a Gray-code rank), sort both by rank, compute exact softmax
+ * attention inside aligned diagonal blocks of the sorted order, estimate the softmax normaliser by adding
+ * a rescaled uniform sample of m key columns to the exact block row sums, approximate the product with V
+ * from the same sampled columns, and merge the two parts. The causal variant (same page, one-line summary
+ * and "Limitations") splits recursively into a causal upper-left half, a causal lower-right half and a
+ * non-causal off-diagonal block, with exact causal attention below a base size, and merges the parts in
+ * log space.
+ *
+ * Conventions for every entry point:
+ *   - Return value: HA_OK (0) or a negative ha_status. Argument errors are detected on the host before
+ *     anything is enqueued; the text of the last error is available from hyper_attn_last_error().
+ *   - Device pointers are plain CUDA device addresses owned by the caller; the library never frees them.
+ *     Host pointers are ordinary host memory owned by the caller (page-locked memory makes copies faster).
+ *   - Tensors Q, K, V, O are dense row-major [batch, heads, n, d] with element type given by the options
+ *     (bf16 by default), 16-byte aligned base addresses.
+ *   - A handle is used by one host thread at a time. Work is enqueued on the handle's stream
+ *     (hyper_attn_set_options) and runs asynchronously unless stated otherwise.
+ *   - There is no CPU fallback: without a usable sm_100 device the calls fail with HA_ERR_CUDA or
+ *     HA_ERR_UNSUPPORTED.
+ */
+#ifndef HYPER_ATTN_H
+#define HYPER_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define HA_API __attribute__((visibility("default")))
+#else
+#define HA_API
+#endif
+
+typedef struct hyper_attn_s *hyper_attn_t;
+
+typedef enum {
+    HA_OK = 0,
+    HA_ERR_INVALID_ARG = -1,  /* a shape, pointer or option is outside what the method accepts */
+    HA_ERR_UNSUPPORTED = -2,  /* valid for the method but not implemented on this device or dtype */
+    HA_ERR_CUDA = -3,         /* a CUDA runtime call failed (message in hyper_attn_last_error) */
+    HA_ERR_OOM = -4,          /* workspace allocation failed */
+    HA_ERR_TIMEOUT = -5       /* a bounded device-side wait gave up (reported by hyper_attn_status) */
+} ha_status;
+
+typedef enum { HA_DTYPE_BF16 = 0, HA_DTYPE_FP32 = 1 } ha_dtype;
+
+/* Attention kernel family. AUTO: tensor-core (tcgen05) kernels for bf16 inputs, SIMT fp32 kernels for
+ * fp32 inputs. SIMT: SIMT fp32 kernels for any input type. TC: tensor-core kernels (bf16 only). */
+typedef enum { HA_KERNEL_AUTO = 0, HA_KERNEL_SIMT = 1, HA_KERNEL_TC = 2 } ha_kernel;
+
+typedef struct {
+    int dtype;            /* ha_dtype of Q, K, V. Default HA_DTYPE_BF16. */
+    int out_dtype;        /* ha_dtype of O, or -1 for "same as dtype". Default -1. */
+    int64_t batch;        /* B >= 1; the problems are the B*heads (batch, head) pairs. Default 1. */
+    int64_t causal_base;  /* c: size below which the causal recursion is exact causal attention.
+                             Default 4096. Causal calls need n = c * 2^L (L >= 0) or n <= c. */
+    void *stream;         /* cudaStream_t to enqueue on; NULL = the legacy default stream. */
+    int kernel;           /* ha_kernel. Default HA_KERNEL_AUTO. */
+    int debug_captures;   /* 1: also store the per-row log normaliser (HA_DBG_LSE, non-causal). Default 0. */
+} ha_options;
+
+/* Create a handle bound to CUDA device `device`. The handle owns a grow-only device workspace (ranks,
+ * permutations, per-level partial results, the draws) and a small page-locked staging buffer.
+ * Fails with HA_ERR_CUDA if the device cannot be used, HA_ERR_UNSUPPORTED if it is not sm_100. */
+HA_API int hyper_attn_create(hyper_attn_t *out, int device);
+
+/* Replace the handle's options (copied). Invalid values return HA_ERR_INVALID_ARG and keep the old ones. */
+HA_API int hyper_attn_set_options(hyper_attn_t h, const ha_options *opt);
+
+/* Fill *opt with the defaults listed above. */
+HA_API void hyper_attn_default_options(ha_options *opt);
+
+/*
+ * HyperAttention forward on device memory: O = approx softmax(Q K^T) V for every (batch, head).
+ *   Q, K, V (in), O (out): device pointers, [batch, heads, n, d]; O must not alias Q, K or V.
+ *   No softmax scale is applied inside exp: callers fold it into Q and K (e.g. both times d^-1/4).
+ *   n      rows per head; n % min(block, n) == 0.
+ *   d      head dimension, 64 or 128.
+ *   block  b: sorted rows per diagonal block (b' = min(b, N) for a problem of N rows).
+ *   m      columns sampled uniformly without replacement per problem, 0 <= m <= N of every problem.
+ *   r      LSH projections (hash bits), 0 <= r <= 16; r = 0 puts every row in one bucket.
+ *   causal 0: one problem of n queries and n keys. 1: the recursive causal variant with the handle's
+ *          causal_base; every off-diagonal problem has N >= causal_base rows and needs b | N, m <= N.
+ *   seed   drives the projection matrix and the column samples (see hyper_attn_draw).
+ * Enqueued on the handle's stream; returns after enqueueing. Argument errors return synchronously and
+ * enqueue nothing. The workspace is reused by the next call on the same handle (stream-ordered).
+ */
+HA_API int hyper_attn_forward(hyper_attn_t h, const void *Q, const void *K, const void *V, void *O,
+                       int64_t n, int d, int heads, int block, int m, int r, int causal, uint64_t seed);
+
+/*
+ * Same computation with HOST buffers: copies Q, K, V to handle-owned device buffers, runs the forward
+ * pass, copies O back and waits for the stream. Returns when O is valid on the host. Page-locked host
+ * memory is copied asynchronously; pageable memory is staged by the CUDA runtime.
+ */
+HA_API int hyper_attn_forward_host(hyper_attn_t h, const void *Q, const void *K, const void *V, void *O,
+                            int64_t n, int d, int heads, int block, int m, int r, int causal, uint64_t seed);
+
+/*
+ * The random draws the forward pass makes for these arguments, computed on the host:
+ *   P_out  [d][r] float: projection matrix, i.i.d. N(0,1) (Philox4x64-10 + Box-Muller), one per call,
+ *          shared by Q and K, all heads and all causal nodes. May be NULL.
+ *   S_out  [bh][nodes][m] int32 (bh = batch*heads): ascending column indices in [0, N) of each problem.
+ *          nodes = 1 (non-causal) or 2^L - 1 (causal; node k is heap node k+1: root 1, children 2i, 2i+1).
+ *          May be NULL.
+ * Host-only, no device needed.
+ */
+HA_API int hyper_attn_draw(uint64_t seed, int d, int r, int64_t bh, int64_t n, int m, int causal, int64_t base,
+                    float *P_out, int32_t *S_out);
+
+/* Number of causal levels L (0 for non-causal) and sample sets per problem for these arguments;
+ * returns HA_ERR_INVALID_ARG for an invalid causal shape. */
+HA_API int hyper_attn_levels(int64_t n, int causal, int64_t base, int *levels_out, int64_t *nodes_out);
+
+/* Debug captures of the last forward call on this handle, copied to host memory after synchronising
+ * the handle's stream. `level` selects the sort level (0 for non-causal, 1..L for causal). */
+typedef enum {
+    HA_DBG_RANK = 0,   /* uint16 [bh][2][n]: sortLSH rank of each Q row (index 0) and K row (index 1) */
+    HA_DBG_NEAR = 1,   /* uint8  [bh][2][n]: 1 when some projection of the row is below 1e-4 * ||row||  */
+    HA_DBG_PERM = 2,   /* int32  [bh][nodes_l][2][N_l]: sorted position -> local row, Q then K segment   */
+    HA_DBG_INV = 3,    /* int32  [bh][nodes_l][2][N_l]: local row -> sorted position                     */
+    HA_DBG_LSE = 4     /* float  [bh][n]: log of the estimated normaliser of each query row (non-causal) */
+} ha_debug_what;
+HA_API int hyper_attn_debug_copy(hyper_attn_t h, int what, int level, void *host_dst, size_t bytes);
+
+/* Synchronise the handle's stream and report device-side status: HA_OK, HA_ERR_TIMEOUT if a bounded
+ * wait gave up, or HA_ERR_CUDA if the stream holds an error. Clears the device status word. */
+HA_API int hyper_attn_status(hyper_attn_t h);
+
+/* Kernel classes for profiling. */
+typedef enum {
+    HA_KC_HASH = 0,        /* sortLSH hash */
+    HA_KC_SORT = 1,        /* counting-sort passes (count, scan, scatter) */
+    HA_KC_ATTN = 2,        /* block + sampled attention of one level, including the gather and the merge */
+    HA_KC_CAUSAL_BASE = 3, /* exact causal leaves and the final log-space merge */
+    HA_KC_COUNT = 4
+} ha_kernel_class;
+
+/* enable = 1: record a CUDA event pair on the handle's stream around every kernel class launch of the
+ * following forward calls; 0: stop recording. Recording adds two event records per launch. */
+HA_API int hyper_attn_profile(hyper_attn_t h, int enable);
+
+/* Synchronise the handle's stream and add, per kernel class (array index = ha_kernel_class, n entries),
+ * the summed device time in milliseconds and the number of kernel launches recorded since the previous
+ * read; then forget the recorded events. ms and launches may be NULL. */
+HA_API int hyper_attn_profile_read(hyper_attn_t h, double *ms, int *launches, int n);
+
+/* Attention kernel family the last forward call used: HA_KERNEL_SIMT or HA_KERNEL_TC (0 before any call). */
+HA_API int hyper_attn_last_kernel(hyper_attn_t h);
+
+/* Kernels launched by the last forward call (for launch accounting). */
+HA_API int hyper_attn_last_launch_count(hyper_attn_t h);
+
+/* Text of the last error on this handle ("" if none). Valid until the next call on the handle. */
+HA_API const char *hyper_attn_last_error(hyper_attn_t h);
+
+/* Release the workspace and the handle. NULL is accepted. Synchronises the handle's stream first. */
+HA_API int hyper_attn_destroy(hyper_attn_t h);
+
+/* Library version as major*10000 + minor*100 + patch. */
+HA_API int hyper_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HYPER_ATTN_H */

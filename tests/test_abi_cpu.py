@@ -1,0 +1,83 @@
+"""Host-side checks of the C-ABI library (no GPU needed): it loads, exports every symbol the header
+declares, its host-side draws equal the oracle's bit for bit, and handle creation fails cleanly without
+a device."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from approximate_long_context_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    import __graft_entry__  # noqa: F401  (build helper)
+    from approximate_long_context_b200 import build
+    build.build()
+    return binding.lib()
+
+
+def declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"^\s*(?:HA_API\s+)?(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(hyper_attn_[a-z_0-9]+)\s*\(", text, re.M)
+    return sorted(set(names))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert len(names) >= 13
+    for name in names:
+        assert hasattr(lib, name), name
+    assert sorted(binding.EXPORTS) == sorted(n for n in names if n in binding.EXPORTS)
+    assert set(names) <= set(binding.EXPORTS) | {"hyper_attn_forward_noalloc"}
+
+
+def test_version(lib):
+    assert lib.hyper_attn_version() >= 100
+
+
+def test_create_without_device_fails_cleanly(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    h = ctypes.c_void_p()
+    rc = lib.hyper_attn_create(ctypes.byref(h), 0)
+    assert rc in (binding.HA_ERR_CUDA, binding.HA_ERR_UNSUPPORTED)
+    assert not h.value
+
+
+@pytest.mark.parametrize("seed,d,r,bh,n,m,causal,base", [
+    (1234, 64, 6, 1, 1024, 64, False, 0),
+    (1237, 64, 8, 3, 131072, 256, False, 0),
+    (1236, 128, 7, 2, 32768, 256, True, 4096),
+    (99, 128, 16, 1, 4096, 0, False, 0),
+    (7, 64, 0, 2, 2048, 17, True, 256),
+])
+def test_draws_match_oracle(lib, ora, seed, d, r, bh, n, m, causal, base):
+    P, S = binding.draw(seed, d, r, bh, n, m, causal=causal, base=base)
+    assert np.array_equal(P.view(np.uint32), ora.draw_projection(seed, d, r).view(np.uint32))
+    L, nodes = binding.levels(n, causal, base) if causal else (0, 1)
+    for b in range(bh):
+        for k in range(nodes):
+            node = k + 1
+            depth = node.bit_length() - 1
+            N = n >> (depth + 1) if causal else n
+            assert np.array_equal(S[b, k], ora.draw_samples(seed, b, node, N, m))
+
+
+def test_levels(lib):
+    assert binding.levels(32768, True, 4096) == (3, 7)
+    assert binding.levels(524288, True, 8192) == (6, 63)
+    assert binding.levels(4096, True, 8192) == (0, 0)
+    with pytest.raises(binding.HAError):
+        binding.levels(3 * 4096, True, 4096)
+    with pytest.raises(binding.HAError):
+        binding.draw(1, 64, 4, 1, 100, 101, causal=False)

@@ -36,7 +36,7 @@ def run_gpu(ha, Qh, Kh, Vh, *, n, d, bh, block, m, r, causal, seed, base=4096, d
             kernel="auto", debug=True):
     Q, K, V = dev_tensor(Qh), dev_tensor(Kh), dev_tensor(Vh)
     O = torch.empty((bh, n, d), dtype=torch.float32 if out_dtype == "fp32" else torch.bfloat16, device="cuda")
-    ha.set_options(dtype=dtype, out_dtype=out_dtype, batch=1, causal_base=base, kernel=kernel,
+    ha.set_options(dtype=dtype, out_dtype=out_dtype, batch=1, causal_base=base or 4096, kernel=kernel,
                    stream=torch.cuda.current_stream().cuda_stream, debug_captures=debug)
     ha.forward(Q, K, V, O, n=n, d=d, heads=bh, block=block, m=m, r=r, causal=causal, seed=seed)
     torch.cuda.synchronize()

@@ -24,7 +24,7 @@ EXPORTS = [
     "hyper_attn_forward_host", "hyper_attn_draw", "hyper_attn_levels", "hyper_attn_debug_copy",
     "hyper_attn_status", "hyper_attn_last_launch_count", "hyper_attn_last_error", "hyper_attn_destroy",
     "hyper_attn_version", "hyper_attn_profile", "hyper_attn_profile_read",
-    "hyper_attn_last_kernel",
+    "hyper_attn_last_kernel", "hyper_attn_forward_noalloc",
 ]
 KERNEL_CLASSES = ["hash", "sort", "attn", "causal_base"]
 
@@ -76,6 +76,7 @@ def lib():
     L.hyper_attn_version.argtypes = []
     L.hyper_attn_profile.argtypes = [vp, ci]
     L.hyper_attn_last_kernel.argtypes = [vp]
+    L.hyper_attn_forward_noalloc.argtypes = [vp, vp, vp, vp, i64, ci, ci, ci, ci, ci, u64, ci, vp]
     L.hyper_attn_profile_read.argtypes = [vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ci), ci]
     _lib = L
     return L

@@ -37,7 +37,7 @@ def test_exports_every_declared_symbol(lib):
     for name in names:
         assert hasattr(lib, name), name
     assert sorted(binding.EXPORTS) == sorted(n for n in names if n in binding.EXPORTS)
-    assert set(names) <= set(binding.EXPORTS) | {"hyper_attn_forward_noalloc"}
+    assert set(names) <= set(binding.EXPORTS)
 
 
 def test_version(lib):

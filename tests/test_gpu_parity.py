@@ -16,6 +16,9 @@ pytestmark = pytest.mark.gpu
 torch = pytest.importorskip("torch")
 
 TOL = {"fp32": 1e-4, "bf16": 2e-3}
+# log of the estimated normaliser: fp32 paths sum fp32 terms; the tensor-core path sums the bf16-rounded
+# probabilities it feeds to the P.V product, so |dL| <= 2^-8 (bf16 unit roundoff) plus fp32 rounding
+LSE_TOL = {"fp32": 1e-4, "bf16": 2.0 ** -8 + 2.0 ** -12}
 
 
 def dev_tensor(a):
@@ -42,6 +45,15 @@ def run_gpu(ha, Qh, Kh, Vh, *, n, d, bh, block, m, r, causal, seed, base=4096, d
     torch.cuda.synchronize()
     assert ha.status() == 0, ha.last_error()
     return O.float().cpu().numpy().astype(np.float64)
+
+
+def tc_shape(n, block, causal, base):
+    """Shapes the tensor-core kernels take: every level's b' = min(b, N) and the causal leaf are multiples
+    of 128."""
+    if not causal:
+        return min(block, n) % 128 == 0
+    levels = binding.levels(n, True, base)[0]
+    return min(base, n) % 128 == 0 and all(min(block, n >> l) % 128 == 0 for l in range(1, levels + 1))
 
 
 def rel_err(a, b):
@@ -92,15 +104,25 @@ CASES = [
     ("causal_d128", 8192, 128, 2, 256, 128, 7, True, 1024, "bf16"),
     ("causal_exact_only", 1024, 64, 2, 64, 32, 6, True, 4096, "bf16"),
     ("causal_fp32", 2048, 64, 1, 64, 64, 6, True, 256, "fp32"),
+    # shapes aimed at the tensor-core kernels: ragged sample chunks, 1- and 3-tile blocks, odd leaves
+    ("tc_m100", 2048, 64, 2, 256, 100, 6, False, 0, "bf16"),
+    ("tc_m200_d128", 2048, 128, 2, 128, 200, 7, False, 0, "bf16"),
+    ("tc_block384", 1536, 64, 2, 384, 64, 5, False, 0, "bf16"),
+    ("tc_m0_d128", 1024, 128, 1, 256, 0, 6, False, 0, "bf16"),
+    ("tc_many_heads", 1024, 64, 16, 256, 128, 6, False, 0, "bf16"),
+    ("tc_causal_leaf384", 1536, 128, 2, 128, 64, 6, True, 384, "bf16"),
+    ("tc_causal_d64", 4096, 64, 2, 256, 256, 8, True, 1024, "bf16"),
 ]
 
 
-@pytest.mark.parametrize("kernel", ["simt", "auto"])
+@pytest.mark.parametrize("kernel", ["simt", "auto", "tc"])
 @pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
 def test_parity_small(ha, case, kernel):
     name, n, d, bh, block, m, r, causal, base, dtype = case
-    if kernel == "auto" and dtype == "fp32":
-        pytest.skip("auto selects the SIMT kernels for fp32")
+    if kernel != "simt" and dtype == "fp32":
+        pytest.skip("the tensor-core kernels take bf16 inputs")
+    if kernel == "tc" and not tc_shape(n, block, causal, base):
+        pytest.skip("shape outside the tensor-core kernels (b' or the causal leaf not a multiple of 128)")
     seed = 1000 + sum(map(ord, name))
     Qh, Kh, Vh = wl.make_inputs(n, d, bh, data_seed=seed, planted=0.05, sinks=causal, dtype=dtype)
     Qf, Kf, Vf = wl.as_f32(Qh), wl.as_f32(Kh), wl.as_f32(Vh)
@@ -113,7 +135,7 @@ def test_parity_small(ha, case, kernel):
         assert e < TOL[dtype], f"head {h}: relative L2 error {e:.3e}"
         if not causal:
             lse = ha.debug_copy("lse", 0, np.float32, bh * n).reshape(bh, n)[h]
-            assert np.max(np.abs(lse - ref["L"])) < (1e-4 if dtype == "fp32" else 1e-3)
+            assert np.max(np.abs(lse - ref["L"])) < LSE_TOL[dtype]
 
 
 def test_bf16_output(ha):

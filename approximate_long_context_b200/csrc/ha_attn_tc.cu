@@ -1,34 +1,41 @@
-// ha_attn_tc.cu -- tensor-core (tcgen05 / TMEM / TMA) attention kernels for bf16 inputs.
+// ha_attn_tc.cu -- tensor-core (tcgen05 / TMEM) attention kernels for bf16 inputs.
 //
 // Two modes share one persistent kernel:
 //
 //  LEVEL: the HyperAttention problem of one level ("HyperAttention: Long-context Attention in Near-Linear
 //  Time", research-map summary, "Approach"). A work item is a pair of 128-query tiles of one sorted block
-//  i. Its key stream is the b'/64 chunks of key block i (exact block part) followed by ceil(m/64) chunks
+//  i. Its key stream is the b'/128 chunks of key block i (exact block part) followed by ceil(m/128) chunks
 //  of sampled columns (uniform sample part). The loader compacts the sample list per item: columns whose
 //  key lies in block i are already counted exactly and are dropped, the rest keep their order and carry
 //  the weight N/m (+ log2(N/m) on the base-2 score); only the tail of the last sample chunk is masked.
-//  Rows are fetched through the sort permutations with TMA tile::gather4 loads straight into
-//  128-byte-swizzled shared memory, so no permuted copy of Q, K or V exists. One online softmax over both
-//  parts gives O = (N1+N2)/(D1+D2); the epilogue writes each row to its original position (merge and
-//  un-permute), or, for causal levels, the fp32 part and its log normaliser.
+//  Rows are read through the sort permutations (the gather) with 16-byte cp.async copies straight into
+//  the 128-byte-swizzled layout the tensor core reads, so no permuted copy of Q, K or V exists. One online
+//  softmax over both parts gives O = (N1+N2)/(D1+D2); the epilogue writes each row to its original position
+//  (the merge and un-permute), or, for causal levels, the fp32 part and its log normaliser.
 //
 //  CAUSAL: exact causal attention inside leaves of c rows (the summary's recursive causal extension: the
 //  base case), merged in log space with the parts of every causal level the row belongs to
 //  ("Limitations": partitioning and merging). A work item is a pair of query tiles of one leaf; query tile
-//  g sees key chunks 0..2g+1, the last two with the inclusive causal mask. Items run heaviest first.
+//  g sees key chunks 0..g, the last one with the inclusive causal mask. Items run heaviest first.
+//
+// Work unit of the MMA and softmax roles: a "pair" (query tile t, key chunk c) of 128 x 128 scores. The
+// pairs of an item run c-major, t-minor. S of pair k lives in TMEM buffer k mod R of a ring of R buffers of
+// 128 columns; the softmax overwrites it with P (bf16, its first 64 columns) and the P.V product reads P
+// from TMEM. The MMA issues S of pair k+R right after P.V of pair k (same buffer, issued in order), so up
+// to R score tiles are in flight while the softmax works. (On this part an M=128, K=16 MMA costs about
+// the same for N = 64 and N = 128, so 128-key chunks halve the cost of the score products.)
 //
 // CTA layout (384 threads, one CTA per SM, persistent):
-//   warp 0      loader: Q tiles, K/V chunks of 64 rows (ring of NST stages), per-item sample list;
-//   warp 1      MMA issuer (lane 0): S = Q K^T into TMEM (two S buffers per tile, so the next chunk's
-//               scores are computed while the softmax works on the current one), O += P V with P in TMEM;
+//   warp 0      K/V loader: 128-row chunks into a ring of NST stages, per-item sample list;
+//   warp 2      Q loader: the two query tiles of an item (QB buffers per tile);
+//   warp 1      MMA issuer (lane 0);
 //   warps 4-7   softmax of tile 0, warps 8-11 softmax of tile 1: a thread owns one query row (TMEM lane),
-//               reads its 64 scores once, keeps the running max and sum, writes P (bf16) over S, rescales O
-//               only when the running max grows by more than 2^8, and runs the epilogue.
-// TMEM (512 columns): S buffers of tile t at [128 t, 128 t + 64) and [128 t + 64, 128 t + 128) (P occupies
-// the first 32 columns of its buffer), O of tile t at [256 + d t, 256 + d t + d).
+//               keeps the running max and sum, rescales O only when the running max grows by more than 2^8,
+//               and runs the epilogue.
+// Loaders copy with cp.async and arrive on the stage barrier when their copies complete.
+// TMEM (512 columns): S ring at [0, 128 R); O of tile t at [128 R + d t, 128 R + d (t + 1)).
 // Every mbarrier wait is bounded; on expiry the kernel sets the status bit, the other warps give up, the
-// loader waits (bounded) for its copies in flight, and TMEM is freed before exit.
+// loaders wait for their copies, the MMA issuer drains the tensor core, and TMEM is freed before exit.
 #include <math.h>
 
 #include "ha_common.cuh"
@@ -41,7 +48,7 @@ namespace {
 using namespace sm100;
 
 constexpr int kThreads = 384;
-constexpr int kKC = 64;                 // keys per chunk
+constexpr int kKC = 128;                // keys per chunk
 constexpr int kMaxLevels = 16;
 constexpr int kMaxSampleList = 1024;    // sampled columns per problem handled by the tensor-core path
 constexpr int kMaxBlock = 1024;         // rows per sorted block handled by the tensor-core path
@@ -76,15 +83,15 @@ struct TcArgs {
 };
 
 struct Item {
-    bool valid[2];
-    int nc[2];            // key chunks of each tile
-    int nc_max;
+    bool v0, v1;          // tile validity
+    int nc0, nc1;         // key chunks of each tile (0 when invalid)
+    int nc_max, npairs;
     // LEVEL
     int64_t prob, blk, bhi, node;
     int pair;
     // CAUSAL
     int64_t leaf_start;   // global row of the leaf's first row (bhi * n + leaf offset)
-    int gt[2];            // query tile index within the leaf
+    int gt0, gt1;         // query tile index within the leaf
 };
 
 __device__ __forceinline__ Item decode(const TcArgs &a, int64_t it) {
@@ -98,11 +105,10 @@ __device__ __forceinline__ Item decode(const TcArgs &a, int64_t it) {
         x.pair = static_cast<int>(rem % a.pairs_per_block);
         x.bhi = x.prob / a.lv.nodes;
         x.node = x.prob % a.lv.nodes;
-        for (int t = 0; t < 2; ++t) {
-            x.valid[t] = x.pair * 2 + t < a.tiles_per_block;
-            x.nc[t] = a.nb + a.ns;
-        }
-        x.nc_max = a.nb + a.ns;
+        x.v0 = x.pair * 2 < a.tiles_per_block;
+        x.v1 = x.pair * 2 + 1 < a.tiles_per_block;
+        x.nc0 = x.v0 ? a.nb + a.ns : 0;
+        x.nc1 = x.v1 ? a.nb + a.ns : 0;
     } else {
         const int64_t per_pair = a.bh * a.nleaves;
         const int pair = a.pairs_per_leaf - 1 - static_cast<int>(it / per_pair);   // heaviest first
@@ -110,91 +116,117 @@ __device__ __forceinline__ Item decode(const TcArgs &a, int64_t it) {
         x.bhi = rem / a.nleaves;
         x.leaf_start = x.bhi * a.n + (rem % a.nleaves) * a.leaf;
         x.pair = pair;
-        x.nc_max = 0;
-        for (int t = 0; t < 2; ++t) {
-            x.gt[t] = pair * 2 + t;
-            x.valid[t] = x.gt[t] < a.tiles_per_leaf;
-            x.nc[t] = x.valid[t] ? 2 * x.gt[t] + 2 : 0;
-            x.nc_max = max(x.nc_max, x.nc[t]);
-        }
+        x.gt0 = pair * 2;
+        x.gt1 = pair * 2 + 1;
+        x.v0 = x.gt0 < a.tiles_per_leaf;
+        x.v1 = x.gt1 < a.tiles_per_leaf;
+        x.nc0 = x.v0 ? x.gt0 + 1 : 0;
+        x.nc1 = x.v1 ? x.gt1 + 1 : 0;
     }
+    x.nc_max = max(x.nc0, x.nc1);
+    x.npairs = x.nc0 + x.nc1;
     return x;
 }
 
+// Position of pair (t, c) in the item's pair order (c-major, t-minor, skipping finished tiles).
+__device__ __forceinline__ int pair_index(const Item &x, int t, int c) {
+    const int mn = min(x.nc0, x.nc1);
+    if (mn == 0) return c;
+    if (c < mn) return 2 * c + t;
+    return 2 * mn + (c - mn);
+}
+
+// Inverse of pair_index.
+__device__ __forceinline__ void pair_tc(const Item &x, int k, int &t, int &c) {
+    const int mn = min(x.nc0, x.nc1);
+    if (mn == 0) { t = x.v0 ? 0 : 1; c = k; return; }
+    if (k < 2 * mn) { t = k & 1; c = k >> 1; return; }
+    t = x.nc0 > x.nc1 ? 0 : 1;
+    c = mn + (k - 2 * mn);
+}
+
 template <int D>
-struct Smem {
-    static constexpr int kSlabs = D / 64;
-    static constexpr int kTileBytes = 128 * D * 2;       // one 128-row Q tile (bf16)
-    static constexpr int kChunkBytes = kKC * D * 2;      // one 64-row K or V chunk
-    static constexpr int kStages = D == 64 ? 8 : 4;
+struct Cfg {
+    static constexpr int R = D == 64 ? 3 : 2;          // S ring buffers
+    static constexpr int QB = D == 64 ? 2 : 1;         // Q buffers per tile
+    static constexpr int NST = D == 64 ? 4 : 2;        // K/V stages
+    static constexpr int kOCol = R * 128;              // first O column
+    static constexpr int kTileBytes = 128 * D * 2;     // 128 rows of bf16 (a Q tile, a K or a V chunk)
     static constexpr int kQ = 0;
-    static constexpr int kK = kQ + 2 * kTileBytes;
-    static constexpr int kV = kK + kStages * kChunkBytes;
-    static constexpr int kList = kV + kStages * kChunkBytes;             // compacted samples of the item
-    static constexpr int kCacheS = kList + kMaxSampleList * 4;           // samples of the current problem
-    static constexpr int kCacheB = kCacheS + kMaxSampleList * 4;         // their sorted key block
-    static constexpr int kKPerm = kCacheB + kMaxSampleList * 4;          // key rows of the item's block
-    static constexpr int kQPerm = kKPerm + kMaxBlock * 4;                // query rows of one tile
+    static constexpr int kK = kQ + 2 * QB * kTileBytes;
+    static constexpr int kV = kK + NST * kTileBytes;
+    static constexpr int kList = kV + NST * kTileBytes;                    // compacted samples of the item
+    static constexpr int kCacheS = kList + kMaxSampleList * 4;             // samples of the current problem
+    static constexpr int kCacheB = kCacheS + kMaxSampleList * 4;           // their sorted key block
+    static constexpr int kKPerm = kCacheB + kMaxSampleList * 4;            // key rows of the item's block
+    static constexpr int kQPerm = kKPerm + kMaxBlock * 4;                  // query rows of one tile
     static constexpr int kWord = kQPerm + 128 * 4;
-    static constexpr int kBars = kWord + kStages * 4 + 64;   // keep 8-byte alignment with slack
-    static constexpr int bQFull = 0, bQEmpty = 2, bKVFull = 4,
-                         bKVEmpty = bKVFull + kStages, bWordFull = bKVEmpty + kStages, bSFull = bWordFull + kStages,
-                         bPFull = bSFull + 4, bOReady = bPFull + 4, bOFinal = bOReady + 2, bOFree = bOFinal + 2,
+    static constexpr int kBars = kWord + NST * 4 + 64;
+    static constexpr int bQFull = 0, bQEmpty = bQFull + 2 * QB, bKVFull = bQEmpty + 2 * QB,
+                         bKVEmpty = bKVFull + NST, bWordFull = bKVEmpty + NST, bSFull = bWordFull + NST,
+                         bPFull = bSFull + R, bOReady = bPFull + R, bOFinal = bOReady + 4, bOFree = bOFinal + 2,
                          bDrain = bOFree + 2, kNumBars = bDrain + 1;
     static constexpr int kTmemSlot = kBars + kNumBars * 8;
     static constexpr int kAbort = kTmemSlot + 4;
     static constexpr int kBytes = kAbort + 4;
     static_assert(kBars % 8 == 0, "mbarriers need 8-byte alignment");
+    static_assert(kOCol + 2 * D <= 512, "TMEM budget");
 };
 
 __device__ __forceinline__ void flag_status(int *status) {
     if (status) atomicOr(status, kStatusTimeout);
 }
 
+// byte offset of 16-byte piece j of row `row` inside a 128-row, 128-byte-swizzled tile (slab s = 64 columns)
+__device__ __forceinline__ uint32_t swz(int slab, int row, int j) {
+    return static_cast<uint32_t>(slab * (128 * 128) + row * 128 + ((j ^ (row & 7)) << 4));
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
-    using L = Smem<D>;
+    using C = Cfg<D>;
     extern __shared__ unsigned char smem_raw[];
     const uint32_t raw_addr = smem_addr(smem_raw);
     const uint32_t pad = (1024u - (raw_addr & 1023u)) & 1023u;
     unsigned char *sm = smem_raw + pad;
     const uint32_t sbase = raw_addr + pad;
-    auto bar = [&](int i) -> uint32_t { return sbase + L::kBars + 8u * static_cast<uint32_t>(i); };
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::kAbort);
-    int *words = reinterpret_cast<int *>(sm + L::kWord);
-    int32_t *slist = reinterpret_cast<int32_t *>(sm + L::kList);
+    auto bar = [&](int i) -> uint32_t { return sbase + C::kBars + 8u * static_cast<uint32_t>(i); };
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + C::kAbort);
+    int *words = reinterpret_cast<int *>(sm + C::kWord);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 32) {
+        for (int i = 0; i < 2 * C::QB; ++i) {
+            mbar_init(bar(C::bQFull + i), 32);     // the Q loader's lanes (copy completion)
+            mbar_init(bar(C::bQEmpty + i), 1);
+        }
+        for (int s = 0; s < C::NST; ++s) {
+            mbar_init(bar(C::bKVFull + s), 32);    // the K/V loader's lanes (copy completion)
+            mbar_init(bar(C::bKVEmpty + s), 1);
+            mbar_init(bar(C::bWordFull + s), 1);
+        }
+        for (int b = 0; b < C::R; ++b) {
+            mbar_init(bar(C::bSFull + b), 1);
+            mbar_init(bar(C::bPFull + b), 128);
+        }
+        for (int i = 0; i < 4; ++i) mbar_init(bar(C::bOReady + i), 1);
         for (int t = 0; t < 2; ++t) {
-            mbar_init(bar(L::bQFull + t), 32);     // the Q loader warp
-            mbar_init(bar(L::bQEmpty + t), 1);
-            mbar_init(bar(L::bOReady + t), 1);
-            mbar_init(bar(L::bOFinal + t), 1);
-            mbar_init(bar(L::bOFree + t), 128);
-            for (int b = 0; b < 2; ++b) {
-                mbar_init(bar(L::bSFull + 2 * t + b), 1);
-                mbar_init(bar(L::bPFull + 2 * t + b), 128);
-            }
+            mbar_init(bar(C::bOFinal + t), 1);
+            mbar_init(bar(C::bOFree + t), 128);
         }
-        for (int s = 0; s < L::kStages; ++s) {
-            mbar_init(bar(L::bKVFull + s), 32);    // the K/V loader warp
-            mbar_init(bar(L::bKVEmpty + s), 1);
-            mbar_init(bar(L::bWordFull + s), 1);
-        }
-        mbar_init(bar(L::bDrain), 1);
+        mbar_init(bar(C::bDrain), 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
     if (warp == 0) {
-        tmem_alloc(sbase + L::kTmemSlot, 512);
+        tmem_alloc(sbase + C::kTmemSlot, 512);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sm + L::kTmemSlot);
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sm + C::kTmemSlot);
 
     // LEVEL items all cost the same: each CTA takes a contiguous range, so consecutive items share a problem
     // and its cached samples. CAUSAL items are ordered heaviest first and dealt round-robin.
@@ -210,249 +242,219 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
         stride = gridDim.x;
     }
 
-    if (warp == 0 || warp == 2) {
-        // ------------------------------------------------------------------ loaders
-        // warp 2 copies the Q tiles of each item, warp 0 streams the K/V chunks. Rows move as 16-byte cp.async
-        // copies, PPR lanes per row, into the 128-byte-swizzled layout the tensor core reads (16-byte piece j
-        // of row r sits at piece j ^ (r & 7)); when a warp's copies have landed it fences them to the async
-        // proxy and its 32 lanes arrive on the stage's barrier.
-        constexpr int PPR = D / 8;             // 16-byte pieces per row
-        constexpr int RPI = 32 / PPR;          // rows per warp instruction
-        const int rsub = lane / PPR, piece = lane % PPR;
-        const int slab = piece >> 3, jp = piece & 7;
+    constexpr int PPR = D / 8;             // 16-byte pieces per row
+    constexpr int RPI = 32 / PPR;          // rows per warp instruction
+
+    if (warp == 2) {
+        // ------------------------------------------------------------------ Q loader
+        const int rsub = lane / PPR, piece = lane % PPR, slab = piece >> 3, jp = piece & 7;
+        int32_t *qperm = reinterpret_cast<int32_t *>(sm + C::kQPerm);
+        int qc0 = 0, qc1 = 0;
         bool ok = true;
-        if (warp == 2) {
-            int32_t *qperm = reinterpret_cast<int32_t *>(sm + L::kQPerm);
-            int qcnt0 = 0, qcnt1 = 0;
-            for (int64_t it = first; it < last && ok; it += stride) {
-                const Item x = decode(a, it);
+        for (int64_t it = first; it < last && ok; it += stride) {
+            const Item x = decode(a, it);
 #pragma unroll
-                for (int t = 0; t < 2; ++t) {
-                    if (!ok || !x.valid[t]) continue;
-                    int &qc = t == 0 ? qcnt0 : qcnt1;
-                    if (qc > 0 && !mbar_wait(bar(L::bQEmpty + t), (qc - 1) & 1, abort_flag)) { ok = false; continue; }
-                    const uint32_t base = sbase + L::kQ + t * L::kTileBytes;
-                    int64_t qbase;
-                    const bool through_perm = a.mode == MODE_LEVEL;
-                    if (through_perm) {
-                        // the tile's 128 query rows, one 16-byte load per lane, staged in shared memory
-                        const int32_t *pq = a.perm + (x.prob * 2) * a.lv.seg_len + x.blk * a.lv.bp + (x.pair * 2 + t) * 128;
-                        __syncwarp();
-                        reinterpret_cast<int4 *>(qperm)[lane] = reinterpret_cast<const int4 *>(pq)[lane];
-                        __syncwarp();
-                        qbase = x.bhi * a.n + x.node * a.lv.node_len + a.lv.q_off;
-                    } else {
-                        qbase = x.leaf_start + x.gt[t] * 128;
-                    }
-#pragma unroll 8
-                    for (int r0 = 0; r0 < 128; r0 += RPI) {
-                        const int row = r0 + rsub;
-                        const int64_t grow = qbase + (through_perm ? qperm[row] : row);
-                        cp_async16(base + slab * 16384 + row * 128 + ((jp ^ (row & 7)) << 4), a.Q + grow * D + piece * 8);
-                    }
-                    cp_commit();
-                    cp_wait<0>();
-                    fence_proxy_async_smem();
-                    mbar_arrive(bar(L::bQFull + t));
-                    ++qc;
+            for (int t = 0; t < 2; ++t) {
+                if (!ok || !(t == 0 ? x.v0 : x.v1)) continue;
+                int &qc = t == 0 ? qc0 : qc1;
+                const int qb = qc % C::QB;
+                const int use = qc / C::QB;
+                if (use > 0 && !mbar_wait(bar(C::bQEmpty + t * C::QB + qb), (use - 1) & 1, abort_flag)) {
+                    ok = false;
+                    continue;
                 }
-            }
-        } else {
-            const unsigned lt_mask = (1u << lane) - 1u;
-            int32_t *cache_s = reinterpret_cast<int32_t *>(sm + L::kCacheS);
-            int32_t *cache_b = reinterpret_cast<int32_t *>(sm + L::kCacheB);
-            int32_t *kperm = reinterpret_cast<int32_t *>(sm + L::kKPerm);
-            int64_t cached_prob = -1;
-            int64_t g = 0;
-            // commit groups whose barrier arrival is still owed (oldest first); a chunk's arrival is made
-            // once kLag newer groups have been issued, or when the stream drains
-            constexpr int kLag = 2;
-            uint32_t f0 = 0, f1 = 0, f2 = 0;
-            int fn = 0;
-            auto push = [&](uint32_t b) {
-                cp_commit();
-                if (fn == 0) f0 = b; else if (fn == 1) f1 = b; else f2 = b;
-                ++fn;
-                if (fn > kLag) {
-                    cp_wait<kLag>();
-                    fence_proxy_async_smem();
-                    mbar_arrive(f0);
-                    f0 = f1;
-                    f1 = f2;
-                    --fn;
-                }
-            };
-            for (int64_t it = first; it < last && ok; it += stride) {
-                const Item x = decode(a, it);
-                // compacted sample list of this item: the sampled columns whose key lies outside block blk,
-                // in sample order (from the per-problem cache of samples and their sorted blocks)
-                int cnt = 0;
-                int64_t kbase = 0;
-                const int32_t *pk = nullptr;
-                if (a.mode == MODE_LEVEL) {
-                    kbase = x.bhi * a.n + x.node * a.lv.node_len;
-                    const int32_t *pkg = a.perm + (x.prob * 2 + 1) * a.lv.seg_len + x.blk * a.lv.bp;
+                const uint32_t base = sbase + C::kQ + (t * C::QB + qb) * C::kTileBytes;
+                int64_t qbase;
+                const bool through_perm = a.mode == MODE_LEVEL;
+                if (through_perm) {
+                    // the tile's 128 query rows: one 16-byte load per lane, staged in shared memory
+                    const int32_t *pq = a.perm + (x.prob * 2) * a.lv.seg_len + x.blk * a.lv.bp + (x.pair * 2 + t) * 128;
                     __syncwarp();
-                    for (int i = lane; i < a.lv.bp / 4; i += 32)
-                        reinterpret_cast<int4 *>(kperm)[i] = reinterpret_cast<const int4 *>(pkg)[i];
-                    pk = kperm;
-                    if (a.ns > 0) {
-                        if (x.prob != cached_prob) {
-                            const int32_t *Sp = a.S + (x.bhi * a.nodes_total + (a.lv.heap0 + x.node - 1)) * a.m;
-                            const int32_t *ik = a.inv + (x.prob * 2 + 1) * a.lv.seg_len;
-                            __syncwarp();
-                            for (int u = lane; u < a.m; u += 32) cache_s[u] = Sp[u];
-                            __syncwarp();
-                            for (int u = lane; u < a.m; u += 32) cache_b[u] = ik[cache_s[u]] / a.lv.bp;
-                            cached_prob = x.prob;
-                        }
-                        __syncwarp();
-                        for (int base = 0; base < a.m; base += 32) {
-                            const int u = base + lane;
-                            const bool keep = u < a.m && cache_b[u] != x.blk;
-                            const unsigned bal = __ballot_sync(0xffffffffu, keep);
-                            if (keep) slist[cnt + __popc(bal & lt_mask)] = cache_s[u];
-                            cnt += __popc(bal);
-                        }
-                    }
+                    reinterpret_cast<int4 *>(qperm)[lane] = reinterpret_cast<const int4 *>(pq)[lane];
                     __syncwarp();
+                    qbase = x.bhi * a.n + x.node * a.lv.node_len + a.lv.q_off;
+                } else {
+                    qbase = x.leaf_start + static_cast<int64_t>(t == 0 ? x.gt0 : x.gt1) * 128;
                 }
-                for (int c = 0; c < x.nc_max; ++c, ++g) {
-                    const int slot = static_cast<int>(g % L::kStages);
-                    const int64_t round = g / L::kStages;
-                    if (round > 0 && !mbar_wait(bar(L::bKVEmpty + slot), (round - 1) & 1, abort_flag)) { ok = false; break; }
-                    int valid_cols = kKC;
-                    int kind;   // 0: block chunk (through the key permutation), 1: sample chunk, 2: contiguous
-                    int u0 = 0;
-                    if (a.mode == MODE_LEVEL) {
-                        if (c < a.nb) {
-                            kind = 0;
-                        } else {
-                            kind = 1;
-                            u0 = (c - a.nb) * kKC;
-                            valid_cols = min(kKC, max(0, cnt - u0));
-                        }
-                    } else {
-                        kind = 2;
-                    }
-                    if (lane == 0) {
-                        words[slot] = valid_cols;
-                        mbar_arrive(bar(L::bWordFull + slot));
-                    }
-                    const uint32_t kb = sbase + L::kK + slot * L::kChunkBytes;
-                    const uint32_t vb = sbase + L::kV + slot * L::kChunkBytes;
-                    const int64_t cbase = a.mode == MODE_LEVEL ? kbase : x.leaf_start + static_cast<int64_t>(c) * kKC;
 #pragma unroll 8
-                    for (int r0 = 0; r0 < kKC; r0 += RPI) {
-                        const int row = r0 + rsub;
-                        int32_t loc;
-                        if (kind == 0) loc = pk[c * kKC + row];
-                        else if (kind == 1) loc = u0 + row < cnt ? slist[u0 + row] : 0;
-                        else loc = row;
-                        const int64_t goff = (cbase + loc) * D + piece * 8;
-                        const uint32_t off = slab * (kKC * 128) + row * 128 + ((jp ^ (row & 7)) << 4);
-                        cp_async16(kb + off, a.K + goff);
-                        cp_async16(vb + off, a.V + goff);
-                    }
-                    push(bar(L::bKVFull + slot));
+                for (int r0 = 0; r0 < 128; r0 += RPI) {
+                    const int row = r0 + rsub;
+                    const int64_t grow = qbase + (through_perm ? qperm[row] : row);
+                    cp_async16(base + swz(slab, row, jp), a.Q + grow * D + piece * 8);
                 }
+                cp_async_arrive(bar(C::bQFull + t * C::QB + qb));
+                ++qc;
             }
-            // owed arrivals: every copy lands before the CTA moves on or exits
-            cp_wait<0>();
-            fence_proxy_async_smem();
-            if (fn > 0) mbar_arrive(f0);
-            if (fn > 1) mbar_arrive(f1);
-            if (fn > 2) mbar_arrive(f2);
         }
+        cp_wait<0>();
+        if (!ok) flag_status(a.status);
+    } else if (warp == 0) {
+        // ------------------------------------------------------------------ K/V loader
+        const int rsub = lane / PPR, piece = lane % PPR, slab = piece >> 3, jp = piece & 7;
+        const unsigned lt_mask = (1u << lane) - 1u;
+        int32_t *slist = reinterpret_cast<int32_t *>(sm + C::kList);
+        int32_t *cache_s = reinterpret_cast<int32_t *>(sm + C::kCacheS);
+        int32_t *cache_b = reinterpret_cast<int32_t *>(sm + C::kCacheB);
+        int32_t *kperm = reinterpret_cast<int32_t *>(sm + C::kKPerm);
+        int64_t cached_prob = -1;
+        int64_t g = 0;
+        bool ok = true;
+        for (int64_t it = first; it < last && ok; it += stride) {
+            const Item x = decode(a, it);
+            // key rows of block blk and the compacted sample list of this item: the sampled columns whose key
+            // lies outside block blk, in sample order (from the per-problem cache of samples and their blocks)
+            int cnt = 0;
+            int64_t kbase = 0;
+            if (a.mode == MODE_LEVEL) {
+                kbase = x.bhi * a.n + x.node * a.lv.node_len;
+                const int32_t *pkg = a.perm + (x.prob * 2 + 1) * a.lv.seg_len + x.blk * a.lv.bp;
+                __syncwarp();
+                for (int i = lane; i < a.lv.bp / 4; i += 32)
+                    reinterpret_cast<int4 *>(kperm)[i] = reinterpret_cast<const int4 *>(pkg)[i];
+                if (a.ns > 0) {
+                    if (x.prob != cached_prob) {
+                        const int32_t *Sp = a.S + (x.bhi * a.nodes_total + (a.lv.heap0 + x.node - 1)) * a.m;
+                        const int32_t *ik = a.inv + (x.prob * 2 + 1) * a.lv.seg_len;
+                        __syncwarp();
+                        for (int u = lane; u < a.m; u += 32) cache_s[u] = Sp[u];
+                        __syncwarp();
+                        for (int u = lane; u < a.m; u += 32) cache_b[u] = ik[cache_s[u]] / a.lv.bp;
+                        cached_prob = x.prob;
+                    }
+                    __syncwarp();
+                    for (int base = 0; base < a.m; base += 32) {
+                        const int u = base + lane;
+                        const bool keep = u < a.m && cache_b[u] != x.blk;
+                        const unsigned bal = __ballot_sync(0xffffffffu, keep);
+                        if (keep) slist[cnt + __popc(bal & lt_mask)] = cache_s[u];
+                        cnt += __popc(bal);
+                    }
+                }
+                __syncwarp();
+            }
+            for (int c = 0; c < x.nc_max; ++c, ++g) {
+                const int slot = static_cast<int>(g % C::NST);
+                const int64_t round = g / C::NST;
+                if (round > 0 && !mbar_wait(bar(C::bKVEmpty + slot), (round - 1) & 1, abort_flag)) { ok = false; break; }
+                int valid_cols = kKC;
+                int kind;   // 0: block chunk (through the key permutation), 1: sample chunk, 2: contiguous
+                int u0 = 0;
+                if (a.mode == MODE_LEVEL) {
+                    if (c < a.nb) {
+                        kind = 0;
+                    } else {
+                        kind = 1;
+                        u0 = (c - a.nb) * kKC;
+                        valid_cols = min(kKC, max(0, cnt - u0));
+                    }
+                } else {
+                    kind = 2;
+                }
+                if (lane == 0) {
+                    words[slot] = valid_cols;
+                    mbar_arrive(bar(C::bWordFull + slot));
+                }
+                const uint32_t kb = sbase + C::kK + slot * C::kTileBytes;
+                const uint32_t vb = sbase + C::kV + slot * C::kTileBytes;
+                const int64_t cbase = a.mode == MODE_LEVEL ? kbase : x.leaf_start + static_cast<int64_t>(c) * kKC;
+#pragma unroll 8
+                for (int r0 = 0; r0 < kKC; r0 += RPI) {
+                    const int row = r0 + rsub;
+                    int32_t loc;
+                    if (kind == 0) loc = kperm[c * kKC + row];
+                    else if (kind == 1) loc = u0 + row < cnt ? slist[u0 + row] : 0;
+                    else loc = row;
+                    const int64_t goff = (cbase + loc) * D + piece * 8;
+                    const uint32_t off = swz(slab, row, jp);
+                    cp_async16(kb + off, a.K + goff);
+                    cp_async16(vb + off, a.V + goff);
+                }
+                cp_async_arrive(bar(C::bKVFull + slot));
+            }
+        }
+        cp_wait<0>();
         if (!ok) flag_status(a.status);
     } else if (warp == 1) {
         // ------------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16(128, kKC, false, false);
             constexpr uint32_t idesc_pv = idesc_bf16(128, D, false, true);
-            int64_t g = 0;
-            int qcnt0 = 0, qcnt1 = 0, ocnt0 = 0, ocnt1 = 0, pb00 = 0, pb01 = 0, pb10 = 0, pb11 = 0;
+            // descriptors are built once; an MMA only adds a byte offset >> 4 to the start-address field
+            const uint64_t dq0 = smem_desc(sbase + C::kQ, 16, 1024);
+            const uint64_t dk0 = smem_desc(sbase + C::kK, 16, 1024);
+            const uint64_t dv0 = smem_desc(sbase + C::kV, 128 * 128, 1024);
+            int64_t g = 0, kp = 0;   // chunks and pairs before the current item
+            int qc0 = 0, qc1 = 0, oc0 = 0, oc1 = 0;
             bool ok = true;
-            auto tS = [&](int t, int b) -> uint32_t { return tmem + t * 128 + b * 64; };
-            auto issue_s = [&](int t, int b, int slot) {
-                const uint32_t qa = sbase + L::kQ + t * L::kTileBytes;
-                const uint32_t ka = sbase + L::kK + slot * L::kChunkBytes;
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t qoff = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    const uint32_t koff = (kk >> 2) * (kKC * 128) + (kk & 3) * 32;
-                    mma_ss(tS(t, b), smem_desc(qa + qoff, 16, 1024), smem_desc(ka + koff, 16, 1024), idesc_qk,
-                           kk > 0 ? 1u : 0u);
-                }
-            };
-            auto wait_k = [&](int64_t gc) -> bool {
-                return mbar_wait(bar(L::bKVFull + static_cast<int>(gc % L::kStages)), (gc / L::kStages) & 1, abort_flag);
-            };
             for (int64_t it = first; it < last && ok; it += stride) {
                 const Item x = decode(a, it);
-                // first two score chunks of each tile
-                for (int c0 = 0; c0 < 2 && ok; ++c0) {
-                    if (c0 >= x.nc_max) break;
-                    if (!wait_k(g + c0)) { ok = false; break; }
-#pragma unroll
-                    for (int t = 0; t < 2; ++t) {
-                        if (!x.valid[t] || c0 >= x.nc[t]) continue;
-                        if (c0 == 0) {
-                            int &qc = t == 0 ? qcnt0 : qcnt1;
-                            if (!mbar_wait(bar(L::bQFull + t), qc & 1, abort_flag)) { ok = false; break; }
-                            ++qc;
-                        }
-                        tc_fence_after();
-                        issue_s(t, c0, static_cast<int>((g + c0) % L::kStages));
-                        mma_commit(bar(L::bSFull + 2 * t + c0));
-                        if (c0 == x.nc[t] - 1) mma_commit(bar(L::bQEmpty + t));
-                    }
+                int qb0 = 0, qb1 = 0;
+                if (x.v0) {
+                    qb0 = qc0 % C::QB;
+                    if (!mbar_wait(bar(C::bQFull + qb0), (qc0 / C::QB) & 1, abort_flag)) { ok = false; break; }
+                    ++qc0;
                 }
-                for (int c = 0; c < x.nc_max && ok; ++c) {
+                if (x.v1) {
+                    qb1 = qc1 % C::QB;
+                    if (!mbar_wait(bar(C::bQFull + C::QB + qb1), (qc1 / C::QB) & 1, abort_flag)) { ok = false; break; }
+                    ++qc1;
+                }
+                auto issue_s = [&](int k) -> bool {
+                    int t, c;
+                    pair_tc(x, k, t, c);
                     const int64_t gc = g + c;
-                    const int slot = static_cast<int>(gc % L::kStages);
-                    if (!mbar_wait(bar(L::bKVFull + slot), (gc / L::kStages) & 1, abort_flag)) { ok = false; break; }
-                    const int b = c & 1;
+                    const int slot = static_cast<int>(gc % C::NST);
+                    if (!mbar_wait(bar(C::bKVFull + slot), (gc / C::NST) & 1, abort_flag)) return false;
+                    tc_fence_after();
+                    const int buf = static_cast<int>((kp + k) % C::R);
+                    const int qb = t == 0 ? qb0 : qb1;
+                    const uint64_t dq = dq0 + static_cast<uint64_t>(((t * C::QB + qb) * C::kTileBytes) >> 4);
+                    const uint64_t dk = dk0 + static_cast<uint64_t>((slot * C::kTileBytes) >> 4);
 #pragma unroll
-                    for (int t = 0; t < 2; ++t) {
-                        if (!ok || !x.valid[t] || c >= x.nc[t]) continue;
-                        int &pc = t == 0 ? (b ? pb01 : pb00) : (b ? pb11 : pb10);
-                        if (!mbar_wait(bar(L::bPFull + 2 * t + b), pc & 1, abort_flag)) { ok = false; continue; }
-                        ++pc;
-                        const int oc = t == 0 ? ocnt0 : ocnt1;
-                        if (c == 0 && oc > 0 && !mbar_wait(bar(L::bOFree + t), (oc - 1) & 1, abort_flag)) { ok = false; continue; }
-                        tc_fence_after();
-                        const uint32_t va = sbase + L::kV + slot * L::kChunkBytes;
-#pragma unroll
-                        for (int kk = 0; kk < kKC / 16; ++kk)
-                            mma_ts(tmem + 256 + t * D, tS(t, b) + kk * 8, smem_desc(va + kk * 2048, kKC * 128, 1024),
-                                   idesc_pv, (c > 0 || kk > 0) ? 1u : 0u);
-                        mma_commit(bar(L::bOReady + t));
-                        if (c == x.nc[t] - 1) mma_commit(bar(L::bOFinal + t));
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint64_t off = static_cast<uint64_t>(((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4);
+                        mma_ss(tmem + buf * 128, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
                     }
-                    if (!ok) break;
-                    // chunk c is consumed once these P.V products finish: release its stage before waiting for
-                    // chunk c + 2, whose arrival may depend on that stage
-                    mma_commit(bar(L::bKVEmpty + slot));
+                    mma_commit(bar(C::bSFull + buf));
+                    // last score tile of this query tile in this item: its Q buffer may be refilled
+                    if (c == (t == 0 ? x.nc0 : x.nc1) - 1) mma_commit(bar(C::bQEmpty + t * C::QB + qb));
+                    return true;
+                };
+                const int np = x.npairs;
+                for (int k = 0; k < np && k < C::R && ok; ++k) ok = issue_s(k);
+                for (int k = 0; k < np && ok; ++k) {
+                    int t, c;
+                    pair_tc(x, k, t, c);
+                    const int64_t gc = g + c;
+                    const int slot = static_cast<int>(gc % C::NST);
+                    const int buf = static_cast<int>((kp + k) % C::R);
+                    if (!mbar_wait(bar(C::bPFull + buf), ((kp + k) / C::R) & 1, abort_flag)) { ok = false; break; }
+                    const int oc = t == 0 ? oc0 : oc1;
+                    if (c == 0 && oc > 0 && !mbar_wait(bar(C::bOFree + t), (oc - 1) & 1, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    // V of chunk c arrived with K (one barrier per stage), which S of this pair waited for
+                    const uint64_t dv = dv0 + static_cast<uint64_t>((slot * C::kTileBytes) >> 4);
+                    const uint32_t od = tmem + C::kOCol + t * D;
 #pragma unroll
-                    for (int t = 0; t < 2; ++t) {
-                        if (!ok || !x.valid[t] || c + 2 >= x.nc[t]) continue;
-                        if (!wait_k(gc + 2)) { ok = false; continue; }
-                        tc_fence_after();
-                        issue_s(t, b, static_cast<int>((gc + 2) % L::kStages));
-                        mma_commit(bar(L::bSFull + 2 * t + b));
-                        if (c + 2 == x.nc[t] - 1) mma_commit(bar(L::bQEmpty + t));
-                    }
-                    if (!ok) break;
+                    for (int kk = 0; kk < kKC / 16; ++kk)
+                        mma_ts(od, tmem + buf * 128 + kk * 8, dv + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv,
+                               (c > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(bar(C::bOReady + 2 * t + (c & 1)));
+                    if (c == (t == 0 ? x.nc0 : x.nc1) - 1) mma_commit(bar(C::bOFinal + t));
+                    // the chunk's stage is free once every tile that uses it has issued its P.V
+                    const bool last_user = t == 1 || c >= x.nc1;
+                    if (last_user) mma_commit(bar(C::bKVEmpty + slot));
+                    if (k + C::R < np) ok = issue_s(k + C::R);
                 }
                 g += x.nc_max;
-                if (x.valid[0]) ++ocnt0;
-                if (x.valid[1]) ++ocnt1;
+                kp += np;
+                if (x.v0) ++oc0;
+                if (x.v1) ++oc1;
             }
             if (!ok) flag_status(a.status);
-            mma_commit(bar(L::bDrain));   // every MMA issued so far completes before TMEM is released
+            mma_commit(bar(C::bDrain));   // every MMA issued so far completes before TMEM is released
             volatile int no_abort = 0;
-            mbar_wait(bar(L::bDrain), 0, &no_abort, 200000000ull);
+            mbar_wait(bar(C::bDrain), 0, &no_abort, 200000000ull);
         }
         __syncwarp();
     } else if (warp >= 4) {
@@ -461,16 +463,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
         const int q = warp & 3;                      // TMEM lane quarter
         const int r = q * 32 + lane;                 // row within the tile
         const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
-        const uint32_t tO = trow + 256 + t * D;
-        int64_t g = 0;
-        int sb0 = 0, sb1 = 0, pvcnt = 0, fin = 0;
+        const uint32_t tO = trow + C::kOCol + t * D;
+        int64_t kp = 0, g = 0;
+        int hp0 = 0, hp1 = 0, fin = 0;               // P handoffs per chunk parity; epilogues done
         bool ok = true;
         for (int64_t it = first; it < last && ok; it += stride) {
             const Item x = decode(a, it);
-            const bool my_valid = t == 0 ? x.valid[0] : x.valid[1];
-            const int my_nc = t == 0 ? x.nc[0] : x.nc[1];
-            const int my_gt = t == 0 ? x.gt[0] : x.gt[1];
-            if (!my_valid) { g += x.nc_max; continue; }
+            const bool my_valid = t == 0 ? x.v0 : x.v1;
+            const int my_nc = t == 0 ? x.nc0 : x.nc1;
+            const int my_gt = t == 0 ? x.gt0 : x.gt1;
+            if (!my_valid) { kp += x.npairs; g += x.nc_max; continue; }
             int64_t qloc = 0;
             if (a.mode == MODE_LEVEL) {
                 const int64_t pos = x.blk * a.lv.bp + (x.pair * 2 + t) * 128 + r;
@@ -478,18 +480,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
             }
             float m_run = -INFINITY, l = 0.0f;
             for (int c = 0; c < my_nc; ++c) {
-                const int64_t gc = g + c;
-                const int b = c & 1;
-                const uint32_t tS = trow + t * 128 + b * 64;
-                if (!mbar_wait(bar(L::bSFull + 2 * t + b), (b ? sb1 : sb0) & 1, abort_flag)) { ok = false; break; }
-                if (b) ++sb1; else ++sb0;
-                // column bound: columns > bound are masked (bound >= 63: none)
+                const int64_t k = kp + pair_index(x, t, c);
+                const int buf = static_cast<int>(k % C::R);
+                const uint32_t tS = trow + buf * 128;
+                if (!mbar_wait(bar(C::bSFull + buf), (k / C::R) & 1, abort_flag)) { ok = false; break; }
+                // column bound: columns > bound are masked (bound >= 127: none)
                 int bound = kKC - 1;
                 float w2 = 0.0f;
                 if (a.mode == MODE_LEVEL) {
                     if (c >= a.nb) {
-                        const int slot = static_cast<int>(gc % L::kStages);
-                        if (!mbar_wait(bar(L::bWordFull + slot), (gc / L::kStages) & 1, abort_flag)) { ok = false; break; }
+                        const int64_t gc = g + c;
+                        const int slot = static_cast<int>(gc % C::NST);
+                        if (!mbar_wait(bar(C::bWordFull + slot), (gc / C::NST) & 1, abort_flag)) { ok = false; break; }
                         bound = words[slot] - 1;
                         w2 = a.lw2;
                     }
@@ -497,35 +499,40 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                     bound = my_gt * 128 + r - c * kKC;
                 }
                 tc_fence_after();
-                uint32_t va[32], vb[32];   // scores of columns 0-31 and 32-63 (registers; indices are constants)
-                tmem_ld32(tS, va);
-                tmem_ld32(tS + 32, vb);
-                tmem_ld_wait();
-                if (__any_sync(0xffffffffu, bound < kKC - 1)) {
+                const bool masked = __any_sync(0xffffffffu, bound < kKC - 1);
+                // pass 1: row max, 64 columns at a time (registers stay below the spill limit)
+                float smax = -INFINITY;
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        if (e > bound) va[e] = 0xff800000u;   // -inf
-                        if (e + 32 > bound) vb[e] = 0xff800000u;
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t va[32], vb[32];
+                    tmem_ld32(tS + h * 64, va);
+                    tmem_ld32(tS + h * 64 + 32, vb);
+                    tmem_ld_wait();
+                    if (masked) {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            if (h * 64 + e > bound) va[e] = 0xff800000u;   // -inf
+                            if (h * 64 + 32 + e > bound) vb[e] = 0xff800000u;
+                        }
                     }
-                }
-                float mx0 = __uint_as_float(va[0]), mx1 = __uint_as_float(va[1]);
-                float mx2 = __uint_as_float(vb[0]), mx3 = __uint_as_float(vb[1]);
+                    float mx0 = __uint_as_float(va[0]), mx1 = __uint_as_float(vb[0]);
 #pragma unroll
-                for (int e = 2; e < 32; e += 2) {
-                    mx0 = fmaxf(mx0, __uint_as_float(va[e]));
-                    mx1 = fmaxf(mx1, __uint_as_float(va[e + 1]));
-                    mx2 = fmaxf(mx2, __uint_as_float(vb[e]));
-                    mx3 = fmaxf(mx3, __uint_as_float(vb[e + 1]));
+                    for (int e = 1; e < 32; ++e) {
+                        mx0 = fmaxf(mx0, __uint_as_float(va[e]));
+                        mx1 = fmaxf(mx1, __uint_as_float(vb[e]));
+                    }
+                    smax = fmaxf(smax, fmaxf(mx0, mx1));
                 }
-                const float smax = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
                 const float xmax = smax == -INFINITY ? -INFINITY : fmaf(smax, kLog2e, w2);
                 const float m_new = xmax > m_run + kRescaleLog2 ? xmax : m_run;
                 const bool grow = m_new != m_run;
                 const float alpha = grow ? ex2_approx(m_run - m_new) : 1.0f;   // 0 when m_run = -inf
                 l *= alpha;
                 if (c > 0 && __any_sync(0xffffffffu, grow)) {
-                    // O holds P.V of chunks 0..c-1; the last of them (PV of chunk c-1) may still be running
-                    if (!mbar_wait(bar(L::bOReady + t), (pvcnt - 1) & 1, abort_flag)) ok = false;
+                    // O holds P.V of chunks 0..c-1: wait for the last of them (chunk c-1) before scaling it
+                    const int pp = (c - 1) & 1;
+                    const int use = (pp ? hp1 : hp0) - 1;
+                    if (!mbar_wait(bar(C::bOReady + 2 * t + pp), use & 1, abort_flag)) ok = false;
                     if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
                     tc_fence_after();
 #pragma unroll
@@ -541,29 +548,45 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                 }
                 m_run = m_new;
                 const float off = w2 - m_run;
-                uint32_t pk[32];
                 float l0 = 0.0f, l1 = 0.0f;
+                // pass 2: P = 2^(x - m_run) in bf16 over the first 64 columns of the buffer (keys 0-63 land in
+                // columns 0-31, already read; keys 64-127 in columns 32-63, read by the first half)
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const float p0 = ex2_approx(fmaf(__uint_as_float(va[2 * e]), kLog2e, off));
-                    const float p1 = ex2_approx(fmaf(__uint_as_float(va[2 * e + 1]), kLog2e, off));
-                    const float p2 = ex2_approx(fmaf(__uint_as_float(vb[2 * e]), kLog2e, off));
-                    const float p3 = ex2_approx(fmaf(__uint_as_float(vb[2 * e + 1]), kLog2e, off));
-                    l0 += p0 + p1;
-                    l1 += p2 + p3;
-                    pk[e] = pack_bf16x2(p0, p1);
-                    pk[16 + e] = pack_bf16x2(p2, p3);
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t va[32], vb[32];
+                    tmem_ld32(tS + h * 64, va);
+                    tmem_ld32(tS + h * 64 + 32, vb);
+                    tmem_ld_wait();
+                    if (masked) {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            if (h * 64 + e > bound) va[e] = 0xff800000u;
+                            if (h * 64 + 32 + e > bound) vb[e] = 0xff800000u;
+                        }
+                    }
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float p0 = ex2_approx(fmaf(__uint_as_float(va[2 * e]), kLog2e, off));
+                        const float p1 = ex2_approx(fmaf(__uint_as_float(va[2 * e + 1]), kLog2e, off));
+                        const float p2 = ex2_approx(fmaf(__uint_as_float(vb[2 * e]), kLog2e, off));
+                        const float p3 = ex2_approx(fmaf(__uint_as_float(vb[2 * e + 1]), kLog2e, off));
+                        l0 += p0 + p1;
+                        l1 += p2 + p3;
+                        pk[e] = pack_bf16x2(p0, p1);
+                        pk[16 + e] = pack_bf16x2(p2, p3);
+                    }
+                    tmem_st32(tS + h * 32, pk);
                 }
                 l += l0 + l1;
-                tmem_st32(tS, pk);
                 tmem_st_wait();
                 tc_fence_before();
-                mbar_arrive(bar(L::bPFull + 2 * t + b));
-                ++pvcnt;
+                mbar_arrive(bar(C::bPFull + buf));
+                if (c & 1) ++hp1; else ++hp0;
             }
             if (!ok) break;
             // epilogue: wait for the tile's last P.V of this item, then write the row
-            if (!mbar_wait(bar(L::bOFinal + t), fin & 1, abort_flag)) ok = false;
+            if (!mbar_wait(bar(C::bOFinal + t), fin & 1, abort_flag)) ok = false;
             if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
             ++fin;
             tc_fence_after();
@@ -615,10 +638,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                 }
             } else {
                 // exact causal leaf part merged with the level parts of this row (log space)
-                const int64_t orow = x.leaf_start + my_gt * 128 + r;
+                const int64_t orow = x.leaf_start + static_cast<int64_t>(my_gt) * 128 + r;
                 const int64_t bhi = x.bhi, qrow = orow - bhi * a.n;
                 const int64_t half_n = a.n / 2;
-                // the level parts this row belongs to: level l holds the row when it lies in the lower half of its node
+                // the level parts this row belongs to: level l holds the row when it lies in the lower half of
+                // its node
                 auto part_index = [&](int lvl, int64_t &dense) -> bool {
                     const int64_t len = a.n >> (lvl - 1), half = len / 2, within = qrow % len;
                     if (within < half) return false;
@@ -681,7 +705,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                 }
             }
             tc_fence_before();
-            mbar_arrive(bar(L::bOFree + t));
+            mbar_arrive(bar(C::bOFree + t));
+            kp += x.npairs;
             g += x.nc_max;
         }
         if (!ok) flag_status(a.status);
@@ -708,7 +733,7 @@ int launch_tc(const void *Q, const void *K, const void *V, TcArgs args, cudaStre
     args.Q = static_cast<const uint16_t *>(Q);
     args.K = static_cast<const uint16_t *>(K);
     args.V = static_cast<const uint16_t *>(V);
-    const size_t smem = Smem<D>::kBytes + 1024;
+    const size_t smem = Cfg<D>::kBytes + 1024;
     auto kern = attn_tc_kernel<D>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
         return -1;

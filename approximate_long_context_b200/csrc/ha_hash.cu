@@ -9,143 +9,184 @@
 // chains over k = 0..d-1 from +0, so the sign decision is reproducible bit for bit. A row whose smallest
 // |x.P_j| is below 1e-4 * ||x||_2 is flagged as near zero.
 //
-// Layout: one CTA hashes 128 consecutive rows of the combined index g = ((bh*2 + which)*n + row)
-// (which 0 = Q, 1 = K). The rows are staged in shared memory with 16-byte cp.async copies (coalesced;
-// the row stride is padded by 16 bytes so that the per-thread row reads do not collide on banks), then
-// each thread runs the chains of one row. P is staged transposed ([j][k]) so that the k-loop reads it as
-// broadcast float4 loads.
+// Layout: persistent CTAs of 128 threads walk tiles of 128 consecutive rows of the combined index
+// g = ((bh*2 + which)*n + row) (which 0 = Q, 1 = K), one row per thread. Tiles are double-buffered in
+// shared memory: the 16-byte cp.async copies of tile i+1 (coalesced; row stride padded by 16 bytes against
+// bank conflicts) are in flight while tile i is hashed. P sits in shared memory as [d][r4] (r rounded up to
+// a multiple of 4); for each k a thread reads P[k][0..r) with broadcast 16-byte loads and advances each
+// projection's chain by one fused multiply-add.
 #include "ha_common.cuh"
 #include "ha_internal.h"
 
 namespace ha {
 namespace {
 
-constexpr int kRowsPerCta = 128;
+constexpr int kRows = 128;
 
-template <int D, int DTYPE>
-__global__ void __launch_bounds__(kRowsPerCta) hash_kernel(const void *__restrict__ Q, const void *__restrict__ K,
-                                                           int64_t n, int64_t total_rows,
-                                                           const float *__restrict__ P, int r,
-                                                           uint16_t *__restrict__ rank, uint8_t *__restrict__ near) {
+template <int D, int DTYPE, int R4>
+__global__ void __launch_bounds__(kRows) hash_kernel(const void *__restrict__ Q, const void *__restrict__ K,
+                                                     int64_t n, int64_t total_rows, const float *__restrict__ P,
+                                                     int r, uint16_t *__restrict__ rank, uint8_t *__restrict__ near) {
     constexpr int ESZ = DTYPE == 0 ? 2 : 4;
     constexpr int ROW_BYTES = D * ESZ;
     constexpr int STRIDE = ROW_BYTES + 16;
     constexpr int CHUNKS = ROW_BYTES / 16;
+    constexpr int EPC = 16 / ESZ;          // elements per 16-byte chunk
+    // R4: r rounded up to a multiple of 4 (compile time, so the unrolled loops carry no conditions); the
+    // padded projections multiply zero columns of P and are ignored.
     extern __shared__ __align__(16) unsigned char smem[];
-    float *PT = reinterpret_cast<float *>(smem);                       // [kMaxR][D]
-    unsigned char *tile = smem + kMaxR * D * sizeof(float);            // [kRowsPerCta][STRIDE]
+    float *Ps = reinterpret_cast<float *>(smem);                               // [D][max(R4, 4)]
+    constexpr int PS = R4 > 0 ? R4 : 4;
+    unsigned char *tiles = smem + D * PS * sizeof(float);                      // [2][kRows][STRIDE]
 
     const int tid = threadIdx.x;
-    const int64_t g0 = static_cast<int64_t>(blockIdx.x) * kRowsPerCta;
-
-    for (int i = tid; i < r * D; i += kRowsPerCta) {
-        const int j = i / D, k = i % D;
-        PT[j * D + k] = P[k * r + j];
+    for (int i = tid; i < D * PS; i += kRows) {
+        const int k = i / PS, j = i % PS;
+        Ps[i] = j < r ? P[k * r + j] : 0.0f;
     }
-    for (int c = tid; c < kRowsPerCta * CHUNKS; c += kRowsPerCta) {
-        const int row = c / CHUNKS, ch = c % CHUNKS;
-        const int64_t g = g0 + row;
-        if (g < total_rows) {
-            const int64_t which = (g / n) & 1, bhi = g / (2 * n), rr = g % n;
+    const int64_t ntiles = (total_rows + kRows - 1) / kRows;
+
+    // stage one tile: 16-byte pieces, CHUNKS consecutive threads per row. The tile's first row is located
+    // once (segment = g / n); later rows step forward, wrapping into the next segment at most 128 / n times.
+    auto stage = [&](int64_t tile, int buf) {
+        unsigned char *dst = tiles + buf * (kRows * STRIDE);
+        const int64_t g0 = tile * kRows;
+        const int64_t seg0 = g0 / n, rr0 = g0 - seg0 * n;
+        const int ch = tid % CHUNKS;
+        for (int row = tid / CHUNKS; row < kRows; row += kRows / CHUNKS) {
+            if (g0 + row >= total_rows) break;
+            int64_t seg = seg0, rr = rr0 + row;
+            while (rr >= n) { rr -= n; ++seg; }
+            const int64_t which = seg & 1, bhi = seg >> 1;
             const unsigned char *src = static_cast<const unsigned char *>(which ? K : Q) +
                                        ((bhi * n + rr) * D) * ESZ + ch * 16;
-            cp_async_16(tile + row * STRIDE + ch * 16, src);
+            cp_async_16(dst + row * STRIDE + ch * 16, src);
         }
-    }
-    cp_async_commit();
-    cp_async_wait<0>();
-    __syncthreads();
+        cp_async_commit();
+    };
 
-    const int64_t g = g0 + tid;
-    if (g >= total_rows) return;
-    const unsigned char *row = tile + tid * STRIDE;
+    int64_t tile = blockIdx.x;
+    if (tile < ntiles) stage(tile, 0);
+    int buf = 0;
+    for (; tile < ntiles; tile += gridDim.x, buf ^= 1) {
+        const int64_t next = tile + gridDim.x;
+        if (next < ntiles) {
+            stage(next, buf ^ 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();   // tile `buf` (and P on the first pass) visible to every thread
 
-    float acc[kMaxR];
+        const int64_t g = tile * kRows + tid;
+        if (g < total_rows) {
+            const unsigned char *row = tiles + buf * (kRows * STRIDE) + tid * STRIDE;
+            float acc[R4 > 0 ? R4 : 1];
 #pragma unroll
-    for (int j = 0; j < kMaxR; ++j) acc[j] = 0.0f;
-    float nrm2 = 0.0f;
-
-#pragma unroll 1
-    for (int h = 0; h < D / 64; ++h) {
-        float x[64];
+            for (int j = 0; j < R4; ++j) acc[j] = 0.0f;
+            float nrm2 = 0.0f;
+#pragma unroll 2
+            for (int c = 0; c < CHUNKS; ++c) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(row + c * 16);
+                float x[EPC];
+                if (DTYPE == 0) {
+                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int c = 0; c < 64 * ESZ / 16; ++c) {
-            const uint4 v = *reinterpret_cast<const uint4 *>(row + h * 64 * ESZ + c * 16);
-            if (DTYPE == 0) {
-                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    x[c * 8 + 2 * e] = __uint_as_float(w[e] << 16);
-                    x[c * 8 + 2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+                    for (int e = 0; e < 4; ++e) {
+                        x[2 * e] = __uint_as_float(w[e] << 16);
+                        x[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+                    }
+                } else {
+                    x[0] = __uint_as_float(v.x);
+                    x[1] = __uint_as_float(v.y);
+                    x[2] = __uint_as_float(v.z);
+                    x[3] = __uint_as_float(v.w);
                 }
-            } else {
-                x[c * 4 + 0] = __uint_as_float(v.x);
-                x[c * 4 + 1] = __uint_as_float(v.y);
-                x[c * 4 + 2] = __uint_as_float(v.z);
-                x[c * 4 + 3] = __uint_as_float(v.w);
-            }
-        }
 #pragma unroll
-        for (int k = 0; k < 64; ++k) nrm2 = __fmaf_rn(x[k], x[k], nrm2);
+                for (int e = 0; e < EPC; ++e) {
+                    const int k = c * EPC + e;
+                    nrm2 = __fmaf_rn(x[e], x[e], nrm2);
+                    const float4 *pk = reinterpret_cast<const float4 *>(Ps + k * PS);
 #pragma unroll
-        for (int j = 0; j < kMaxR; ++j) {
-            if (j < r) {
-                const float4 *pj = reinterpret_cast<const float4 *>(PT + j * D + h * 64);
-#pragma unroll
-                for (int k4 = 0; k4 < 16; ++k4) {
-                    const float4 p = pj[k4];
-                    acc[j] = __fmaf_rn(x[4 * k4 + 0], p.x, acc[j]);
-                    acc[j] = __fmaf_rn(x[4 * k4 + 1], p.y, acc[j]);
-                    acc[j] = __fmaf_rn(x[4 * k4 + 2], p.z, acc[j]);
-                    acc[j] = __fmaf_rn(x[4 * k4 + 3], p.w, acc[j]);
+                    for (int q4 = 0; q4 < R4 / 4; ++q4) {
+                        const float4 p = pk[q4];
+                        acc[4 * q4 + 0] = __fmaf_rn(x[e], p.x, acc[4 * q4 + 0]);
+                        acc[4 * q4 + 1] = __fmaf_rn(x[e], p.y, acc[4 * q4 + 1]);
+                        acc[4 * q4 + 2] = __fmaf_rn(x[e], p.z, acc[4 * q4 + 2]);
+                        acc[4 * q4 + 3] = __fmaf_rn(x[e], p.w, acc[4 * q4 + 3]);
+                    }
                 }
             }
-        }
-    }
-
-    const float thr = __fmul_rn(1e-4f, __fsqrt_rn(nrm2));
-    uint32_t code = 0;
-    bool flag = false;
+            const float thr = __fmul_rn(1e-4f, __fsqrt_rn(nrm2));
+            uint32_t code = 0;
+            bool flag = false;
 #pragma unroll
-    for (int j = 0; j < kMaxR; ++j) {
-        if (j < r) {
-            code |= (acc[j] > 0.0f ? 1u : 0u) << j;
-            flag |= fabsf(acc[j]) < thr;
+            for (int j = 0; j < R4; ++j) {
+                if (j < r) {
+                    code |= (acc[j] > 0.0f ? 1u : 0u) << j;
+                    flag |= fabsf(acc[j]) < thr;
+                }
+            }
+            // inverse Gray code: prefix XOR of all right shifts (16-bit codes)
+            uint32_t g2 = code;
+            g2 ^= g2 >> 1;
+            g2 ^= g2 >> 2;
+            g2 ^= g2 >> 4;
+            g2 ^= g2 >> 8;
+            rank[g] = static_cast<uint16_t>(g2);
+            near[g] = flag ? 1 : 0;
         }
+        __syncthreads();   // everyone is done with tile `buf` before it is refilled
     }
-    // inverse Gray code: prefix XOR of all right shifts (16-bit codes)
-    uint32_t g2 = code;
-    g2 ^= g2 >> 1;
-    g2 ^= g2 >> 2;
-    g2 ^= g2 >> 4;
-    g2 ^= g2 >> 8;
-    rank[g] = static_cast<uint16_t>(g2);
-    near[g] = flag ? 1 : 0;
 }
 
-template <int D, int DTYPE>
+int num_sms_hash() {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms;
+}
+
+template <int D, int DTYPE, int R4>
 int launch_hash_t(const void *Q, const void *K, int64_t bh, int64_t n, const float *P, int r, uint16_t *rank,
                   uint8_t *near, cudaStream_t st) {
     constexpr int ESZ = DTYPE == 0 ? 2 : 4;
-    const size_t smem = kMaxR * D * sizeof(float) + kRowsPerCta * (D * ESZ + 16);
-    auto kern = hash_kernel<D, DTYPE>;
+    const size_t smem = D * (R4 > 0 ? R4 : 4) * sizeof(float) + 2 * kRows * (D * ESZ + 16);
+    auto kern = hash_kernel<D, DTYPE, R4>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
         return -1;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kRows, smem) != cudaSuccess || per_sm < 1)
+        per_sm = 1;
     const int64_t total = 2 * bh * n;
-    const int64_t grid = (total + kRowsPerCta - 1) / kRowsPerCta;
-    kern<<<static_cast<unsigned>(grid), kRowsPerCta, smem, st>>>(Q, K, n, total, P, r, rank, near);
+    const int64_t ntiles = (total + kRows - 1) / kRows;
+    const int64_t slots = static_cast<int64_t>(num_sms_hash()) * per_sm;
+    const int64_t grid = ntiles < slots ? ntiles : slots;
+    kern<<<static_cast<unsigned>(grid), kRows, smem, st>>>(Q, K, n, total, P, r, rank, near);
     return cudaPeekAtLastError() == cudaSuccess ? 1 : -1;
+}
+
+template <int D, int DTYPE>
+int launch_hash_r(const void *Q, const void *K, int64_t bh, int64_t n, const float *P, int r, uint16_t *rank,
+                  uint8_t *near, cudaStream_t st) {
+    switch ((r + 3) / 4) {
+        case 0: return launch_hash_t<D, DTYPE, 0>(Q, K, bh, n, P, r, rank, near, st);
+        case 1: return launch_hash_t<D, DTYPE, 4>(Q, K, bh, n, P, r, rank, near, st);
+        case 2: return launch_hash_t<D, DTYPE, 8>(Q, K, bh, n, P, r, rank, near, st);
+        case 3: return launch_hash_t<D, DTYPE, 12>(Q, K, bh, n, P, r, rank, near, st);
+        default: return launch_hash_t<D, DTYPE, 16>(Q, K, bh, n, P, r, rank, near, st);
+    }
 }
 
 }  // namespace
 
+// P: [d][r] float in device memory.
 int launch_hash(const void *Q, const void *K, int dtype, int64_t bh, int64_t n, int d, const float *P, int r,
                 uint16_t *rank, uint8_t *near, cudaStream_t st) {
-    if (d == 64) return dtype == 0 ? launch_hash_t<64, 0>(Q, K, bh, n, P, r, rank, near, st)
-                                   : launch_hash_t<64, 1>(Q, K, bh, n, P, r, rank, near, st);
-    if (d == 128) return dtype == 0 ? launch_hash_t<128, 0>(Q, K, bh, n, P, r, rank, near, st)
-                                    : launch_hash_t<128, 1>(Q, K, bh, n, P, r, rank, near, st);
-    return -1;
+    if (r < 0 || r > kMaxR || (d != 64 && d != 128)) return -1;
+    if (d == 64) return dtype == 0 ? launch_hash_r<64, 0>(Q, K, bh, n, P, r, rank, near, st)
+                                   : launch_hash_r<64, 1>(Q, K, bh, n, P, r, rank, near, st);
+    return dtype == 0 ? launch_hash_r<128, 0>(Q, K, bh, n, P, r, rank, near, st)
+                      : launch_hash_r<128, 1>(Q, K, bh, n, P, r, rank, near, st);
 }
 
 }  // namespace ha

@@ -26,7 +26,9 @@
 // the same for N = 64 and N = 128, so 128-key chunks halve the cost of the score products.)
 //
 // CTA layout (384 threads, one CTA per SM, persistent):
-//   warp 0      K/V loader: 128-row chunks into a ring of NST stages, per-item sample list;
+//   warp 0      K loader: 128-row chunks into a ring of NST stages, per-item sample list; publishes each
+//               stage's row list for
+//   warp 3      V loader: the V rows of the same chunks;
 //   warp 2      Q loader: the two query tiles of an item (QB buffers per tile);
 //   warp 1      MMA issuer (lane 0);
 //   warps 4-7   softmax of tile 0, warps 8-11 softmax of tile 1: a thread owns one query row (TMEM lane),
@@ -160,10 +162,12 @@ struct Cfg {
     static constexpr int kCacheB = kCacheS + kMaxSampleList * 4;           // their sorted key block
     static constexpr int kKPerm = kCacheB + kMaxSampleList * 4;            // key rows of the item's block
     static constexpr int kQPerm = kKPerm + kMaxBlock * 4;                  // query rows of one tile
-    static constexpr int kWord = kQPerm + 128 * 4;
+    static constexpr int kRows = kQPerm + 128 * 4;                         // global rows of each stage
+    static constexpr int kWord = kRows + NST * 128 * 4;
     static constexpr int kBars = kWord + NST * 4 + 64;
     static constexpr int bQFull = 0, bQEmpty = bQFull + 2 * QB, bKVFull = bQEmpty + 2 * QB,
-                         bKVEmpty = bKVFull + NST, bWordFull = bKVEmpty + NST, bSFull = bWordFull + NST,
+                         bKVEmpty = bKVFull + NST, bWordFull = bKVEmpty + NST, bRowsFull = bWordFull + NST,
+                         bSFull = bRowsFull + NST,
                          bPFull = bSFull + R, bOReady = bPFull + R, bOFinal = bOReady + 4, bOFree = bOFinal + 2,
                          bDrain = bOFree + 2, kNumBars = bDrain + 1;
     static constexpr int kTmemSlot = kBars + kNumBars * 8;
@@ -202,7 +206,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
             mbar_init(bar(C::bQEmpty + i), 1);
         }
         for (int s = 0; s < C::NST; ++s) {
-            mbar_init(bar(C::bKVFull + s), 32);    // the K/V loader's lanes (copy completion)
+            mbar_init(bar(C::bKVFull + s), 64);    // the K and V loader warps' lanes (copy completion)
+            mbar_init(bar(C::bRowsFull + s), 1);
             mbar_init(bar(C::bKVEmpty + s), 1);
             mbar_init(bar(C::bWordFull + s), 1);
         }
@@ -296,6 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
         int32_t *cache_s = reinterpret_cast<int32_t *>(sm + C::kCacheS);
         int32_t *cache_b = reinterpret_cast<int32_t *>(sm + C::kCacheB);
         int32_t *kperm = reinterpret_cast<int32_t *>(sm + C::kKPerm);
+        int32_t *stage_rows = reinterpret_cast<int32_t *>(sm + C::kRows);
         int64_t cached_prob = -1;
         int64_t g = 0;
         bool ok = true;
@@ -354,20 +360,47 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                     words[slot] = valid_cols;
                     mbar_arrive(bar(C::bWordFull + slot));
                 }
-                const uint32_t kb = sbase + C::kK + slot * C::kTileBytes;
-                const uint32_t vb = sbase + C::kV + slot * C::kTileBytes;
+                // the chunk's 128 global rows, published for the V loader
                 const int64_t cbase = a.mode == MODE_LEVEL ? kbase : x.leaf_start + static_cast<int64_t>(c) * kKC;
+                int32_t *rows = stage_rows + slot * 128;
+                for (int row = lane; row < kKC; row += 32) {
+                    int32_t loc;
+                    if (kind == 0) loc = kperm[c * kKC + row];
+                    else if (kind == 1) loc = row + u0 < cnt ? slist[u0 + row] : 0;
+                    else loc = row;
+                    rows[row] = static_cast<int32_t>(cbase + loc);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(C::bRowsFull + slot));
+                const uint32_t kb = sbase + C::kK + slot * C::kTileBytes;
 #pragma unroll 8
                 for (int r0 = 0; r0 < kKC; r0 += RPI) {
                     const int row = r0 + rsub;
-                    int32_t loc;
-                    if (kind == 0) loc = kperm[c * kKC + row];
-                    else if (kind == 1) loc = u0 + row < cnt ? slist[u0 + row] : 0;
-                    else loc = row;
-                    const int64_t goff = (cbase + loc) * D + piece * 8;
-                    const uint32_t off = swz(slab, row, jp);
-                    cp_async16(kb + off, a.K + goff);
-                    cp_async16(vb + off, a.V + goff);
+                    cp_async16(kb + swz(slab, row, jp), a.K + static_cast<int64_t>(rows[row]) * D + piece * 8);
+                }
+                cp_async_arrive(bar(C::bKVFull + slot));
+            }
+        }
+        cp_wait<0>();
+        if (!ok) flag_status(a.status);
+    } else if (warp == 3) {
+        // ------------------------------------------------------------------ V loader
+        // follows the K loader's chunk sequence: waits for each stage's row list, copies the V rows
+        const int rsub = lane / PPR, piece = lane % PPR, slab = piece >> 3, jp = piece & 7;
+        const int32_t *stage_rows = reinterpret_cast<const int32_t *>(sm + C::kRows);
+        int64_t g = 0;
+        bool ok = true;
+        for (int64_t it = first; it < last && ok; it += stride) {
+            const Item x = decode(a, it);
+            for (int c = 0; c < x.nc_max; ++c, ++g) {
+                const int slot = static_cast<int>(g % C::NST);
+                if (!mbar_wait(bar(C::bRowsFull + slot), (g / C::NST) & 1, abort_flag)) { ok = false; break; }
+                const int32_t *rows = stage_rows + slot * 128;
+                const uint32_t vb = sbase + C::kV + slot * C::kTileBytes;
+#pragma unroll 8
+                for (int r0 = 0; r0 < kKC; r0 += RPI) {
+                    const int row = r0 + rsub;
+                    cp_async16(vb + swz(slab, row, jp), a.V + static_cast<int64_t>(rows[row]) * D + piece * 8);
                 }
                 cp_async_arrive(bar(C::bKVFull + slot));
             }

@@ -416,52 +416,87 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
             const uint64_t dq0 = smem_desc(sbase + C::kQ, 16, 1024);
             const uint64_t dk0 = smem_desc(sbase + C::kK, 16, 1024);
             const uint64_t dv0 = smem_desc(sbase + C::kV, 128 * 128, 1024);
-            int64_t g = 0, kp = 0;   // chunks and pairs before the current item
+            // An item in flight: its chunks/pairs offsets, the Q buffer of each tile (-1: not yet waited for)
+            // and how many of its score tiles are already issued. Score tiles run ahead across item
+            // boundaries: once the current item has issued all of its S products, the next item's first
+            // ones go out while the current item's last P.V products wait for their P.
+            struct Flight {
+                Item x;
+                int64_t g, kp;
+                int qb0, qb1;
+                int pre;
+            };
             int qc0 = 0, qc1 = 0, oc0 = 0, oc1 = 0;
             bool ok = true;
+            // wait for (blocking) or test (non-blocking) the Q tile of tile t of item f; false if not ready
+            auto get_q = [&](Flight &f, int t, bool block) -> bool {
+                int &qb = t == 0 ? f.qb0 : f.qb1;
+                if (qb >= 0) return true;
+                int &qc = t == 0 ? qc0 : qc1;
+                const uint32_t b = bar(C::bQFull + t * C::QB + qc % C::QB);
+                const uint32_t par = (qc / C::QB) & 1;
+                if (block) {
+                    if (!mbar_wait(b, par, abort_flag)) { ok = false; return false; }
+                } else if (!mbar_try_wait(b, par)) {
+                    return false;
+                }
+                qb = qc % C::QB;
+                ++qc;
+                return true;
+            };
+            auto issue_s = [&](Flight &f, int k) -> bool {
+                int t, c;
+                pair_tc(f.x, k, t, c);
+                const int64_t gc = f.g + c;
+                const int slot = static_cast<int>(gc % C::NST);
+                if (!mbar_wait(bar(C::bKVFull + slot), (gc / C::NST) & 1, abort_flag)) return false;
+                tc_fence_after();
+                const int buf = static_cast<int>((f.kp + k) % C::R);
+                const int qb = t == 0 ? f.qb0 : f.qb1;
+                const uint64_t dq = dq0 + static_cast<uint64_t>(((t * C::QB + qb) * C::kTileBytes) >> 4);
+                const uint64_t dk = dk0 + static_cast<uint64_t>((slot * C::kTileBytes) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint64_t off = static_cast<uint64_t>(((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4);
+                    mma_ss(tmem + buf * 128, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(bar(C::bSFull + buf));
+                // last score tile of this query tile in this item: its Q buffer may be refilled
+                if (c == (t == 0 ? f.x.nc0 : f.x.nc1) - 1) mma_commit(bar(C::bQEmpty + t * C::QB + qb));
+                ++f.pre;
+                return true;
+            };
+            Flight cur{}, nxt{};
+            bool have_next = false;
+            if (first < last) {
+                cur.x = decode(a, first);
+                cur.g = 0; cur.kp = 0; cur.qb0 = -1; cur.qb1 = -1; cur.pre = 0;
+            }
             for (int64_t it = first; it < last && ok; it += stride) {
-                const Item x = decode(a, it);
-                int qb0 = 0, qb1 = 0;
-                if (x.v0) {
-                    qb0 = qc0 % C::QB;
-                    if (!mbar_wait(bar(C::bQFull + qb0), (qc0 / C::QB) & 1, abort_flag)) { ok = false; break; }
-                    ++qc0;
-                }
-                if (x.v1) {
-                    qb1 = qc1 % C::QB;
-                    if (!mbar_wait(bar(C::bQFull + C::QB + qb1), (qc1 / C::QB) & 1, abort_flag)) { ok = false; break; }
-                    ++qc1;
-                }
-                auto issue_s = [&](int k) -> bool {
+                const Item &x = cur.x;
+                const int np = x.npairs;
+                // score tiles of this item not yet issued by the previous item's look-ahead
+                for (int k = cur.pre; k < np && k < C::R && ok; ++k) {
                     int t, c;
                     pair_tc(x, k, t, c);
-                    const int64_t gc = g + c;
-                    const int slot = static_cast<int>(gc % C::NST);
-                    if (!mbar_wait(bar(C::bKVFull + slot), (gc / C::NST) & 1, abort_flag)) return false;
-                    tc_fence_after();
-                    const int buf = static_cast<int>((kp + k) % C::R);
-                    const int qb = t == 0 ? qb0 : qb1;
-                    const uint64_t dq = dq0 + static_cast<uint64_t>(((t * C::QB + qb) * C::kTileBytes) >> 4);
-                    const uint64_t dk = dk0 + static_cast<uint64_t>((slot * C::kTileBytes) >> 4);
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint64_t off = static_cast<uint64_t>(((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4);
-                        mma_ss(tmem + buf * 128, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
-                    }
-                    mma_commit(bar(C::bSFull + buf));
-                    // last score tile of this query tile in this item: its Q buffer may be refilled
-                    if (c == (t == 0 ? x.nc0 : x.nc1) - 1) mma_commit(bar(C::bQEmpty + t * C::QB + qb));
-                    return true;
-                };
-                const int np = x.npairs;
-                for (int k = 0; k < np && k < C::R && ok; ++k) ok = issue_s(k);
+                    if (!get_q(cur, t, true)) break;
+                    ok = issue_s(cur, k);
+                }
+                have_next = it + stride < last;
+                if (have_next) {
+                    nxt.x = decode(a, it + stride);
+                    nxt.g = cur.g + x.nc_max;
+                    nxt.kp = cur.kp + np;
+                    nxt.qb0 = -1; nxt.qb1 = -1; nxt.pre = 0;
+                }
+                bool look = have_next;   // look-ahead into the next item still possible
                 for (int k = 0; k < np && ok; ++k) {
                     int t, c;
                     pair_tc(x, k, t, c);
-                    const int64_t gc = g + c;
+                    const int64_t gc = cur.g + c;
                     const int slot = static_cast<int>(gc % C::NST);
-                    const int buf = static_cast<int>((kp + k) % C::R);
-                    if (!mbar_wait(bar(C::bPFull + buf), ((kp + k) / C::R) & 1, abort_flag)) { ok = false; break; }
+                    const int buf = static_cast<int>((cur.kp + k) % C::R);
+                    if (!mbar_wait(bar(C::bPFull + buf), ((cur.kp + k) / C::R) & 1, abort_flag)) { ok = false; break; }
                     const int oc = t == 0 ? oc0 : oc1;
                     if (c == 0 && oc > 0 && !mbar_wait(bar(C::bOFree + t), (oc - 1) & 1, abort_flag)) { ok = false; break; }
                     tc_fence_after();
@@ -477,12 +512,27 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                     // the chunk's stage is free once every tile that uses it has issued its P.V
                     const bool last_user = t == 1 || c >= x.nc1;
                     if (last_user) mma_commit(bar(C::bKVEmpty + slot));
-                    if (k + C::R < np) ok = issue_s(k + C::R);
+                    // the ring buffer of pair k is free again: fill it with the score tile R pairs ahead
+                    const int ka = k + C::R;
+                    if (ka < np) {
+                        ok = issue_s(cur, ka);
+                    } else if (look) {
+                        const int kn = ka - np;
+                        if (kn == nxt.pre && kn < nxt.x.npairs) {
+                            int tn, cn;
+                            pair_tc(nxt.x, kn, tn, cn);
+                            // with one Q buffer per tile, the next Q is loaded only after this item's last S:
+                            // take it only if it is already there
+                            if (get_q(nxt, tn, C::QB > 1)) ok = issue_s(nxt, kn);
+                            else look = false;
+                        } else {
+                            look = false;
+                        }
+                    }
                 }
-                g += x.nc_max;
-                kp += np;
                 if (x.v0) ++oc0;
                 if (x.v1) ++oc1;
+                if (have_next) cur = nxt;
             }
             if (!ok) flag_status(a.status);
             mma_commit(bar(C::bDrain));   // every MMA issued so far completes before TMEM is released

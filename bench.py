@@ -34,7 +34,18 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM bytes per launch of a kernel class from an ncu capture, valid only while the source file it was
 # taken from is unchanged (sha256 of the file at capture time).
-TRAFFIC = {}
+TRAFFIC = {
+    # 4-head capture of the 32-head workload (the full one is too large for a multi-pass capture), scaled x8
+    # by the rows processed: attention 205.8 MB read + 42.6 MB written per 4-head launch; hash 134.2 + 5.0 MB.
+    ("attn", "long_bf16_n131072", "tc"): {
+        "file": "ha_attn_tc.cu",
+        "sha256": "9c1760df52f2b25c6a9df7686f44075be3f5e664465c7ffaaf72aeacfd2ed29b",
+        "bytes": 8 * (205_848_064 + 42_623_488)},
+    ("hash", "long_bf16_n131072", "tc"): {
+        "file": "ha_hash.cu",
+        "sha256": "b86668b0d82f1c4fc5e060be3a59b195a331f6726fa6ed7fde3726287ce783fb",
+        "bytes": 8 * (134_234_624 + 4_986_112)},
+}
 
 
 def load_peaks():
@@ -359,11 +370,16 @@ def main():
     ap.add_argument("--workload", default=wl.HEADLINE, choices=sorted(wl.WORKLOADS))
     ap.add_argument("--kernel", default="auto", choices=["auto", "simt", "tc"])
     ap.add_argument("--cpu-heads", type=int, default=32)
+    ap.add_argument("--heads", type=int, default=0,
+                    help="run the workload with this many heads instead of its own (small profiler captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     w = wl.WORKLOADS[args.workload]
+    if args.heads > 0:
+        import dataclasses
+        w = dataclasses.replace(w, heads=args.heads)
     if args.impl == "reference":
         run_reference(args, w)
     else:

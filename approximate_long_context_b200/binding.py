@@ -44,6 +44,7 @@ class Options(ctypes.Structure):
         ("stream", ctypes.c_void_p),
         ("kernel", ctypes.c_int),
         ("debug_captures", ctypes.c_int),
+        ("bh_offset", ctypes.c_int64),
     ]
 
 
@@ -135,7 +136,7 @@ class HyperAttention:
             raise HAError(rc, lib().hyper_attn_last_error(self._h).decode())
 
     def set_options(self, *, dtype="bf16", out_dtype=None, batch=1, causal_base=4096, stream=None,
-                    kernel="auto", debug_captures=False):
+                    kernel="auto", debug_captures=False, bh_offset=0):
         o = Options()
         o.dtype = DTYPES[dtype]
         o.out_dtype = -1 if out_dtype is None else DTYPES[out_dtype]
@@ -144,6 +145,7 @@ class HyperAttention:
         o.stream = stream
         o.kernel = KERNELS[kernel]
         o.debug_captures = int(bool(debug_captures))
+        o.bh_offset = bh_offset
         self._check(lib().hyper_attn_set_options(self._h, ctypes.byref(o)))
         self.options = o
 

@@ -28,7 +28,7 @@ struct hyper_attn_s {
     bool draws_valid = false;
     uint64_t dk_seed = 0;
     int dk_d = 0, dk_r = 0, dk_m = 0, dk_causal = 0;
-    int64_t dk_bh = 0, dk_n = 0, dk_base = 0;
+    int64_t dk_bh = 0, dk_n = 0, dk_base = 0, dk_off = 0;
     // layout of the last forward (for debug copies)
     struct Layout {
         size_t status, P, S, rank, near, lse, perm_tmp, hist, Opart, Lpart, end;
@@ -252,7 +252,7 @@ int ensure_pinned(hyper_attn_t h, size_t bytes) {
 }
 
 // Fill host buffers with the draws of shape s (P: [d][r]; S: [bh][nodes_total][m]).
-int host_draws(uint64_t seed, const Shape &s, float *P, int32_t *S) {
+int host_draws(uint64_t seed, const Shape &s, int64_t bh_offset, float *P, int32_t *S) {
     if (P) ha::draw_projection(seed, s.d, s.r, P);
     if (!S || s.m == 0) return 0;
     std::vector<uint8_t> scratch(static_cast<size_t>(s.n), 0);
@@ -265,7 +265,7 @@ int host_draws(uint64_t seed, const Shape &s, float *P, int32_t *S) {
                 for (int64_t x = node; x > 1; x >>= 1) ++depth;
                 N = s.n >> (depth + 1);
             }
-            if (ha::draw_samples(seed, static_cast<uint64_t>(b), static_cast<uint64_t>(node), N, s.m,
+            if (ha::draw_samples(seed, static_cast<uint64_t>(bh_offset + b), static_cast<uint64_t>(node), N, s.m,
                                  S + (b * s.nodes_total + k) * s.m, scratch.data()))
                 return -1;
         }
@@ -275,7 +275,7 @@ int host_draws(uint64_t seed, const Shape &s, float *P, int32_t *S) {
 
 int upload_draws(hyper_attn_t h, uint64_t seed, const Shape &s, cudaStream_t st) {
     if (h->draws_valid && h->dk_seed == seed && h->dk_d == s.d && h->dk_r == s.r && h->dk_m == s.m &&
-        h->dk_causal == s.causal && h->dk_bh == s.bh && h->dk_n == s.n &&
+        h->dk_causal == s.causal && h->dk_bh == s.bh && h->dk_n == s.n && h->dk_off == h->opt.bh_offset &&
         (!s.causal || h->dk_base == h->opt.causal_base))
         return HA_OK;
     const size_t pbytes = sizeof(float) * ha::kMaxR * 128;
@@ -285,13 +285,13 @@ int upload_draws(hyper_attn_t h, uint64_t seed, const Shape &s, cudaStream_t st)
     HA_CUDA(h, cudaEventSynchronize(h->pin_free));   // the previous upload has left the staging buffer
     float *P = reinterpret_cast<float *>(h->pin);
     int32_t *S = reinterpret_cast<int32_t *>(h->pin + pbytes);
-    if (host_draws(seed, s, P, S)) return fail(h, HA_ERR_INVALID_ARG, "sample draw failed");
+    if (host_draws(seed, s, h->opt.bh_offset, P, S)) return fail(h, HA_ERR_INVALID_ARG, "sample draw failed");
     HA_CUDA(h, cudaMemcpyAsync(h->ws + h->lay.P, P, sizeof(float) * s.d * (s.r ? s.r : 1), cudaMemcpyHostToDevice, st));
     if (sbytes) HA_CUDA(h, cudaMemcpyAsync(h->ws + h->lay.S, S, sbytes, cudaMemcpyHostToDevice, st));
     HA_CUDA(h, cudaEventRecord(h->pin_free, st));
     h->draws_valid = true;
     h->dk_seed = seed; h->dk_d = s.d; h->dk_r = s.r; h->dk_m = s.m; h->dk_causal = s.causal;
-    h->dk_bh = s.bh; h->dk_n = s.n; h->dk_base = h->opt.causal_base;
+    h->dk_bh = s.bh; h->dk_n = s.n; h->dk_base = h->opt.causal_base; h->dk_off = h->opt.bh_offset;
     return HA_OK;
 }
 
@@ -429,6 +429,8 @@ int validate_options(hyper_attn_t h, const ha_options *o) {
     if (o->causal_base < 1) return fail(h, HA_ERR_INVALID_ARG, "causal_base must be >= 1");
     if (o->kernel < HA_KERNEL_AUTO || o->kernel > HA_KERNEL_TC) return fail(h, HA_ERR_INVALID_ARG, "bad kernel");
     if (o->debug_captures != 0 && o->debug_captures != 1) return fail(h, HA_ERR_INVALID_ARG, "bad debug_captures");
+    if (o->bh_offset < 0 || o->bh_offset > (int64_t(1) << 40))
+        return fail(h, HA_ERR_INVALID_ARG, "bh_offset out of range");
     return HA_OK;
 }
 
@@ -453,6 +455,7 @@ void hyper_attn_default_options(ha_options *o) {
     o->stream = nullptr;
     o->kernel = HA_KERNEL_AUTO;
     o->debug_captures = 0;
+    o->bh_offset = 0;
 }
 
 int hyper_attn_version(void) { return kVersion; }
@@ -562,7 +565,7 @@ int hyper_attn_draw(uint64_t seed, int d, int r, int64_t bh, int64_t n, int m, i
     int rc = check_shape(&tmp, n, d == 64 || d == 128 ? d : 64, bh, 1, m, r, causal, &s);
     if (rc) return rc;
     s.d = d;
-    return host_draws(seed, s, P_out, S_out) ? HA_ERR_INVALID_ARG : HA_OK;
+    return host_draws(seed, s, 0, P_out, S_out) ? HA_ERR_INVALID_ARG : HA_OK;
 }
 
 int hyper_attn_levels(int64_t n, int causal, int64_t base, int *levels_out, int64_t *nodes_out) {

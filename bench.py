@@ -220,6 +220,7 @@ def run_ours(args, w: wl.Workload):
     import torch
     import torch.distributed as dist
     from approximate_long_context_b200 import binding
+    from approximate_long_context_b200.shard import max_over_ranks, weak_shard
 
     world, rank, local = dist_setup()
     if world != args.gpus:
@@ -234,7 +235,9 @@ def run_ours(args, w: wl.Workload):
             dist.barrier()
 
     esz = 2 if w.dtype == "bf16" else 4
-    Qh, Kh, Vh = wl.workload_inputs(w)
+    # weak scaling: rank i holds problems [i*bh, (i+1)*bh) of a job of world*bh independent problems
+    sh = weak_shard(w.bh, world, rank)
+    Qh, Kh, Vh = wl.workload_inputs(w, heads=range(sh.offset, sh.offset + sh.count))
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
 
     def pinned(a):
@@ -253,7 +256,7 @@ def run_ours(args, w: wl.Workload):
 
     ha = binding.HyperAttention(local)
     ha.set_options(dtype=w.dtype, batch=w.batch, causal_base=w.base or 4096, stream=stream.cuda_stream,
-                   kernel=args.kernel)
+                   kernel=args.kernel, bh_offset=sh.offset)
     kw = dict(n=w.n, d=w.d, heads=w.heads, block=w.block, m=w.m, r=w.r, causal=w.causal, seed=w.algo_seed)
 
     def step():
@@ -282,10 +285,7 @@ def run_ours(args, w: wl.Workload):
     prof = ha.profile_read()
     assert ha.status() == 0, ha.last_error()
     ms = ev0.elapsed_time(ev1) / args.steps
-    t = torch.tensor([ms], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, dev)
     units = world * w.bh * w.n
     value = units / (ms_max * 1e-3) / 1e6
 
@@ -301,10 +301,8 @@ def run_ours(args, w: wl.Workload):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    te = torch.tensor([e0.elapsed_time(e1) / args.steps], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = units / (float(te.item()) * 1e-3) / 1e6
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
+    e2e_value = units / (e2e_ms * 1e-3) / 1e6
 
     # roofline of the dominant kernel class; sort and attention launch once per level
     peaks, peak_src = load_peaks()

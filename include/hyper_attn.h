@@ -65,6 +65,10 @@ typedef struct {
     void *stream;         /* cudaStream_t to enqueue on; NULL = the legacy default stream. */
     int kernel;           /* ha_kernel. Default HA_KERNEL_AUTO. */
     int debug_captures;   /* 1: also store the per-row log normaliser (HA_DBG_LSE, non-causal). Default 0. */
+    int64_t bh_offset;    /* Global index of this call's first (batch, head) problem, >= 0. The sample draws
+                             of local problem i are those of problem bh_offset + i, so a run split over
+                             several calls or GPUs (each taking a contiguous range of problems) gives the
+                             same result as one call over all problems. Default 0. */
 } ha_options;
 
 /* Create a handle bound to CUDA device `device`. The handle owns a grow-only device workspace (ranks,
@@ -109,6 +113,8 @@ HA_API int hyper_attn_forward_host(hyper_attn_t h, const void *Q, const void *K,
  *   P_out  [d][r] float: projection matrix, i.i.d. N(0,1) (Philox4x64-10 + Box-Muller), one per call,
  *          shared by Q and K, all heads and all causal nodes. May be NULL.
  *   S_out  [bh][nodes][m] int32 (bh = batch*heads): ascending column indices in [0, N) of each problem.
+ *          Problems are numbered from 0; a forward call with option bh_offset = o uses rows o, o+1, ...
+ *          of this array (draw with bh = o + its own problem count).
  *          nodes = 1 (non-causal) or 2^L - 1 (causal; node k is heap node k+1: root 1, children 2i, 2i+1).
  *          May be NULL.
  * Host-only, no device needed.

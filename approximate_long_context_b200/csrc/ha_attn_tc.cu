@@ -82,6 +82,7 @@ struct TcArgs {
     float *lse, *Opart_w, *Lpart_w;
     int *status;
     int64_t items;
+    uint32_t per_outer;    // LEVEL: items per problem; CAUSAL: items per query-tile pair index
 };
 
 struct Item {
@@ -96,27 +97,35 @@ struct Item {
     int gt0, gt1;         // query tile index within the leaf
 };
 
-__device__ __forceinline__ Item decode(const TcArgs &a, int64_t it) {
+// Item index -> item. Item counts, problem counts and their factors are below 2^31 (checked on the host), so the
+// divisions are 32-bit.
+__device__ __forceinline__ Item decode(const TcArgs &a, int64_t it64) {
     Item x{};
+    const uint32_t it = static_cast<uint32_t>(it64);
     if (a.mode == MODE_LEVEL) {
-        const int64_t nblk = a.lv.seg_len / a.lv.bp;
-        const int64_t per_prob = nblk * a.pairs_per_block;
-        x.prob = it / per_prob;
-        const int64_t rem = it % per_prob;
-        x.blk = rem / a.pairs_per_block;
-        x.pair = static_cast<int>(rem % a.pairs_per_block);
-        x.bhi = x.prob / a.lv.nodes;
-        x.node = x.prob % a.lv.nodes;
+        const uint32_t prob = it / a.per_outer;
+        const uint32_t rem = it - prob * a.per_outer;
+        const uint32_t ppb = static_cast<uint32_t>(a.pairs_per_block);
+        const uint32_t blk = rem / ppb;
+        x.prob = prob;
+        x.blk = blk;
+        x.pair = static_cast<int>(rem - blk * ppb);
+        const uint32_t nodes = static_cast<uint32_t>(a.lv.nodes);
+        const uint32_t bhi = prob / nodes;
+        x.bhi = bhi;
+        x.node = prob - bhi * nodes;
         x.v0 = x.pair * 2 < a.tiles_per_block;
         x.v1 = x.pair * 2 + 1 < a.tiles_per_block;
         x.nc0 = x.v0 ? a.nb + a.ns : 0;
         x.nc1 = x.v1 ? a.nb + a.ns : 0;
     } else {
-        const int64_t per_pair = a.bh * a.nleaves;
-        const int pair = a.pairs_per_leaf - 1 - static_cast<int>(it / per_pair);   // heaviest first
-        const int64_t rem = it % per_pair;
-        x.bhi = rem / a.nleaves;
-        x.leaf_start = x.bhi * a.n + (rem % a.nleaves) * a.leaf;
+        const uint32_t po = it / a.per_outer;
+        const int pair = a.pairs_per_leaf - 1 - static_cast<int>(po);   // heaviest first
+        const uint32_t rem = it - po * a.per_outer;
+        const uint32_t nl = static_cast<uint32_t>(a.nleaves);
+        const uint32_t bhi = rem / nl;
+        x.bhi = bhi;
+        x.leaf_start = static_cast<int64_t>(bhi) * a.n + static_cast<int64_t>(rem - bhi * nl) * a.leaf;
         x.pair = pair;
         x.gt0 = pair * 2;
         x.gt1 = pair * 2 + 1;
@@ -151,7 +160,8 @@ template <int D>
 struct Cfg {
     static constexpr int R = D == 64 ? 3 : 2;          // S ring buffers
     static constexpr int QB = D == 64 ? 2 : 1;         // Q buffers per tile
-    static constexpr int NST = D == 64 ? 4 : 2;        // K/V stages
+    static constexpr int NST = D == 64 ? 3 : 2;        // K/V stages
+    static constexpr int SEG = D == 64 ? 128 : 64;     // bytes per row segment of the staged output stores
     static constexpr int kOCol = R * 128;              // first O column
     static constexpr int kTileBytes = 128 * D * 2;     // 128 rows of bf16 (a Q tile, a K or a V chunk)
     static constexpr int kQ = 0;
@@ -164,7 +174,8 @@ struct Cfg {
     static constexpr int kQPerm = kKPerm + kMaxBlock * 4;                  // query rows of one tile
     static constexpr int kRows = kQPerm + 128 * 4;                         // global rows of each stage
     static constexpr int kWord = kRows + NST * 128 * 4;
-    static constexpr int kBars = kWord + NST * 4 + 64;
+    static constexpr int kStage = (kWord + NST * 4 + 64 + 15) / 16 * 16;   // 8 softmax warps x 32 rows x SEG
+    static constexpr int kBars = kStage + 8 * 32 * SEG;
     static constexpr int bQFull = 0, bQEmpty = bQFull + 2 * QB, bKVFull = bQEmpty + 2 * QB,
                          bKVEmpty = bKVFull + NST, bWordFull = bKVEmpty + NST, bRowsFull = bWordFull + NST,
                          bSFull = bRowsFull + NST,
@@ -174,11 +185,74 @@ struct Cfg {
     static constexpr int kAbort = kTmemSlot + 4;
     static constexpr int kBytes = kAbort + 4;
     static_assert(kBars % 8 == 0, "mbarriers need 8-byte alignment");
+    static_assert(kStage % 16 == 0, "16-byte stage pieces");
+    static_assert(kBytes + 1024 <= 232448, "shared memory budget");
     static_assert(kOCol + 2 * D <= 512, "TMEM budget");
 };
 
 __device__ __forceinline__ void flag_status(int *status) {
     if (status) atomicOr(status, kStatusTimeout);
+}
+
+// One SEG-byte segment, at byte offset `off`, of each of the warp's 32 output rows: lane l holds the segment of
+// its own row (16-byte pieces pc[0..SEG/16)) and `drow` points at the start of that row. The segments pass
+// through the warp's shared-memory stage (32 x SEG bytes, pieces XOR-swizzled so that neither the row-wise
+// writes nor the column-wise reads conflict on banks), so that SEG/16 consecutive lanes store one row's SEG
+// contiguous bytes: an instruction touches 32 / (SEG/16) rows instead of 32.
+template <int SEG>
+__device__ __forceinline__ void warp_store_segment(unsigned char *stage, unsigned char *drow, int off,
+                                                   const uint4 (&pc)[SEG / 16], int lane) {
+    constexpr int P = SEG / 16, SH = SEG == 64 ? 1 : 0;
+    __syncwarp();   // the previous segment's reads of the stage are done
+#pragma unroll
+    for (int j = 0; j < P; ++j)
+        *reinterpret_cast<uint4 *>(stage + lane * SEG + ((j ^ ((lane >> SH) & (P - 1))) << 4)) = pc[j];
+    __syncwarp();
+    const int sub = lane / P, piece = lane % P;
+#pragma unroll
+    for (int i = 0; i < P; ++i) {
+        const int row = i * (32 / P) + sub;
+        const uint4 v = *reinterpret_cast<const uint4 *>(stage + row * SEG + ((piece ^ ((row >> SH) & (P - 1))) << 4));
+        unsigned char *rb = reinterpret_cast<unsigned char *>(
+            __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(drow), row));
+        *reinterpret_cast<uint4 *>(rb + off + piece * 16) = v;
+    }
+}
+
+// Write the warp's 32 rows of D output values (bf16 or fp32; lane l owns row l at `drow`). vals(j, v) yields
+// the row's columns [32 j, 32 j + 32) as floats.
+template <int D, int SEG, typename F>
+__device__ __forceinline__ void warp_write_rows(unsigned char *stage, unsigned char *drow, bool bf16, int lane,
+                                                F &&vals) {
+    constexpr int PS = SEG / 16;
+    uint4 seg[PS];
+    if (bf16) {
+#pragma unroll
+        for (int j = 0; j < D / 32; ++j) {
+            float v[32];
+            vals(j, v);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int pi = j * 4 + q;
+                seg[pi % PS] = make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                                          pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+                if (pi % PS == PS - 1) warp_store_segment<SEG>(stage, drow, (pi / PS) * SEG, seg, lane);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < D / 32; ++j) {
+            float v[32];
+            vals(j, v);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int pi = j * 8 + q;
+                seg[pi % PS] = make_uint4(__float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
+                                          __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3]));
+                if (pi % PS == PS - 1) warp_store_segment<SEG>(stage, drow, (pi / PS) * SEG, seg, lane);
+            }
+        }
+    }
 }
 
 // byte offset of 16-byte piece j of row `row` inside a 128-row, 128-byte-swizzled tile (slab s = 64 columns)
@@ -303,7 +377,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
         int32_t *kperm = reinterpret_cast<int32_t *>(sm + C::kKPerm);
         int32_t *stage_rows = reinterpret_cast<int32_t *>(sm + C::kRows);
         int64_t cached_prob = -1;
-        int64_t g = 0;
+        uint32_t g = 0;
         bool ok = true;
         for (int64_t it = first; it < last && ok; it += stride) {
             const Item x = decode(a, it);
@@ -340,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
             }
             for (int c = 0; c < x.nc_max; ++c, ++g) {
                 const int slot = static_cast<int>(g % C::NST);
-                const int64_t round = g / C::NST;
+                const uint32_t round = g / C::NST;
                 if (round > 0 && !mbar_wait(bar(C::bKVEmpty + slot), (round - 1) & 1, abort_flag)) { ok = false; break; }
                 int valid_cols = kKC;
                 int kind;   // 0: block chunk (through the key permutation), 1: sample chunk, 2: contiguous
@@ -388,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
         // follows the K loader's chunk sequence: waits for each stage's row list, copies the V rows
         const int rsub = lane / PPR, piece = lane % PPR, slab = piece >> 3, jp = piece & 7;
         const int32_t *stage_rows = reinterpret_cast<const int32_t *>(sm + C::kRows);
-        int64_t g = 0;
+        uint32_t g = 0;
         bool ok = true;
         for (int64_t it = first; it < last && ok; it += stride) {
             const Item x = decode(a, it);
@@ -422,7 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
             // ones go out while the current item's last P.V products wait for their P.
             struct Flight {
                 Item x;
-                int64_t g, kp;
+                uint32_t g, kp;
                 int qb0, qb1;
                 int pre;
             };
@@ -447,11 +521,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
             auto issue_s = [&](Flight &f, int k) -> bool {
                 int t, c;
                 pair_tc(f.x, k, t, c);
-                const int64_t gc = f.g + c;
+                const uint32_t gc = f.g + c;
                 const int slot = static_cast<int>(gc % C::NST);
                 if (!mbar_wait(bar(C::bKVFull + slot), (gc / C::NST) & 1, abort_flag)) return false;
                 tc_fence_after();
-                const int buf = static_cast<int>((f.kp + k) % C::R);
+                const int buf = static_cast<int>((f.kp + static_cast<uint32_t>(k)) % C::R);
                 const int qb = t == 0 ? f.qb0 : f.qb1;
                 const uint64_t dq = dq0 + static_cast<uint64_t>(((t * C::QB + qb) * C::kTileBytes) >> 4);
                 const uint64_t dk = dk0 + static_cast<uint64_t>((slot * C::kTileBytes) >> 4);
@@ -493,10 +567,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                 for (int k = 0; k < np && ok; ++k) {
                     int t, c;
                     pair_tc(x, k, t, c);
-                    const int64_t gc = cur.g + c;
+                    const uint32_t gc = cur.g + c;
                     const int slot = static_cast<int>(gc % C::NST);
-                    const int buf = static_cast<int>((cur.kp + k) % C::R);
-                    if (!mbar_wait(bar(C::bPFull + buf), ((cur.kp + k) / C::R) & 1, abort_flag)) { ok = false; break; }
+                    const uint32_t kk_all = cur.kp + static_cast<uint32_t>(k);
+                    const int buf = static_cast<int>(kk_all % C::R);
+                    if (!mbar_wait(bar(C::bPFull + buf), (kk_all / C::R) & 1, abort_flag)) { ok = false; break; }
                     const int oc = t == 0 ? oc0 : oc1;
                     if (c == 0 && oc > 0 && !mbar_wait(bar(C::bOFree + t), (oc - 1) & 1, abort_flag)) { ok = false; break; }
                     tc_fence_after();
@@ -547,7 +622,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
         const int r = q * 32 + lane;                 // row within the tile
         const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
         const uint32_t tO = trow + C::kOCol + t * D;
-        int64_t kp = 0, g = 0;
+        uint32_t kp = 0, g = 0;
         int hp0 = 0, hp1 = 0, fin = 0;               // P handoffs per chunk parity; epilogues done
         bool ok = true;
         for (int64_t it = first; it < last && ok; it += stride) {
@@ -563,7 +638,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
             }
             float m_run = -INFINITY, l = 0.0f;
             for (int c = 0; c < my_nc; ++c) {
-                const int64_t k = kp + pair_index(x, t, c);
+                const uint32_t k = kp + static_cast<uint32_t>(pair_index(x, t, c));
                 const int buf = static_cast<int>(k % C::R);
                 const uint32_t tS = trow + buf * 128;
                 if (!mbar_wait(bar(C::bSFull + buf), (k / C::R) & 1, abort_flag)) { ok = false; break; }
@@ -572,7 +647,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                 float w2 = 0.0f;
                 if (a.mode == MODE_LEVEL) {
                     if (c >= a.nb) {
-                        const int64_t gc = g + c;
+                        const uint32_t gc = g + c;
                         const int slot = static_cast<int>(gc % C::NST);
                         if (!mbar_wait(bar(C::bWordFull + slot), (gc / C::NST) & 1, abort_flag)) { ok = false; break; }
                         bound = words[slot] - 1;
@@ -675,48 +750,28 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
             tc_fence_after();
             const float inv_l = 1.0f / l;
             const float Lrow = (m_run + __log2f(l)) * kLn2;   // natural log of the row's normaliser
+            unsigned char *stage = sm + C::kStage + (warp - 4) * (32 * C::SEG);
+            auto o_scaled = [&](float scale) {
+                return [&, scale](int j, float (&v)[32]) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + j * 32, o);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(o[e]) * scale;
+                };
+            };
             if (a.mode == MODE_LEVEL) {
                 const int64_t N = a.lv.seg_len;
                 if (a.lv.level == 0) {
                     const int64_t orow = x.bhi * a.n + a.lv.q_off + x.node * a.lv.node_len + qloc;
-#pragma unroll
-                    for (int j = 0; j < D / 32; ++j) {
-                        uint32_t o[32];
-                        tmem_ld32(tO + j * 32, o);
-                        tmem_ld_wait();
-                        if (a.out_dtype == 0) {
-                            uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(a.O) + orow * D + j * 32);
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                uint4 w;
-                                w.x = pack_bf16x2(__uint_as_float(o[8 * e + 0]) * inv_l, __uint_as_float(o[8 * e + 1]) * inv_l);
-                                w.y = pack_bf16x2(__uint_as_float(o[8 * e + 2]) * inv_l, __uint_as_float(o[8 * e + 3]) * inv_l);
-                                w.z = pack_bf16x2(__uint_as_float(o[8 * e + 4]) * inv_l, __uint_as_float(o[8 * e + 5]) * inv_l);
-                                w.w = pack_bf16x2(__uint_as_float(o[8 * e + 6]) * inv_l, __uint_as_float(o[8 * e + 7]) * inv_l);
-                                dst[e] = w;
-                            }
-                        } else {
-                            float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.O) + orow * D + j * 32);
-#pragma unroll
-                            for (int e = 0; e < 8; ++e)
-                                dst[e] = make_float4(__uint_as_float(o[4 * e]) * inv_l, __uint_as_float(o[4 * e + 1]) * inv_l,
-                                                     __uint_as_float(o[4 * e + 2]) * inv_l, __uint_as_float(o[4 * e + 3]) * inv_l);
-                        }
-                    }
+                    const int esz = a.out_dtype == 0 ? 2 : 4;
+                    unsigned char *drow = static_cast<unsigned char *>(a.O) + orow * D * esz;
+                    warp_write_rows<D, C::SEG>(stage, drow, a.out_dtype == 0, lane, o_scaled(inv_l));
                     if (a.lse) a.lse[orow] = Lrow;
                 } else {
                     const int64_t dense = x.bhi * (a.n / 2) + x.node * N + qloc;
-#pragma unroll
-                    for (int j = 0; j < D / 32; ++j) {
-                        uint32_t o[32];
-                        tmem_ld32(tO + j * 32, o);
-                        tmem_ld_wait();
-                        float4 *dst = reinterpret_cast<float4 *>(a.Opart_w + dense * D + j * 32);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            dst[e] = make_float4(__uint_as_float(o[4 * e]) * inv_l, __uint_as_float(o[4 * e + 1]) * inv_l,
-                                                 __uint_as_float(o[4 * e + 2]) * inv_l, __uint_as_float(o[4 * e + 3]) * inv_l);
-                    }
+                    unsigned char *drow = reinterpret_cast<unsigned char *>(a.Opart_w + dense * D);
+                    warp_write_rows<D, C::SEG>(stage, drow, false, lane, o_scaled(inv_l));
                     a.Lpart_w[dense] = Lrow;
                 }
             } else {
@@ -746,12 +801,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                 }
                 const float inv_tot = 1.0f / tot;
                 const float cb = wb * inv_l * inv_tot;
-#pragma unroll
-                for (int j = 0; j < D / 32; ++j) {
+                auto merged = [&](int j, float (&acc)[32]) {
                     uint32_t o[32];
                     tmem_ld32(tO + j * 32, o);
                     tmem_ld_wait();
-                    float acc[32];
 #pragma unroll
                     for (int e = 0; e < 32; ++e) acc[e] = __uint_as_float(o[e]) * cb;
                     for (int lvl = 1; lvl <= a.levels; ++lvl) {
@@ -768,24 +821,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                             acc[4 * e + 2] += wi * p.z; acc[4 * e + 3] += wi * p.w;
                         }
                     }
-                    if (a.out_dtype == 0) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(a.O) + orow * D + j * 32);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            uint4 w;
-                            w.x = pack_bf16x2(acc[8 * e + 0], acc[8 * e + 1]);
-                            w.y = pack_bf16x2(acc[8 * e + 2], acc[8 * e + 3]);
-                            w.z = pack_bf16x2(acc[8 * e + 4], acc[8 * e + 5]);
-                            w.w = pack_bf16x2(acc[8 * e + 6], acc[8 * e + 7]);
-                            dst[e] = w;
-                        }
-                    } else {
-                        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.O) + orow * D + j * 32);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            dst[e] = make_float4(acc[4 * e], acc[4 * e + 1], acc[4 * e + 2], acc[4 * e + 3]);
-                    }
-                }
+                };
+                const int esz = a.out_dtype == 0 ? 2 : 4;
+                unsigned char *drow = static_cast<unsigned char *>(a.O) + orow * D * esz;
+                warp_write_rows<D, C::SEG>(stage, drow, a.out_dtype == 0, lane, merged);
             }
             tc_fence_before();
             mbar_arrive(bar(C::bOFree + t));
@@ -862,6 +901,8 @@ int launch_attn_tc(const Level &lv, const void *Q, const void *K, const void *V,
     a.Lpart_w = Lpart;
     a.status = status;
     a.items = lv.bh * lv.nodes * (lv.seg_len / lv.bp) * a.pairs_per_block;
+    a.per_outer = static_cast<uint32_t>((lv.seg_len / lv.bp) * a.pairs_per_block);
+    if (a.items >= (int64_t(1) << 31)) return -2;
     return dispatch(d, Q, K, V, a, st);
 }
 
@@ -886,6 +927,8 @@ int launch_causal_base_tc(const void *Q, const void *K, const void *V, int64_t b
     a.out_dtype = out_dtype;
     a.status = status;
     a.items = bh * a.nleaves * a.pairs_per_leaf;
+    a.per_outer = static_cast<uint32_t>(bh * a.nleaves);
+    if (a.items >= (int64_t(1) << 31)) return -2;
     return dispatch(d, Q, K, V, a, st);
 }
 

@@ -209,6 +209,26 @@ METRIC = "HyperAttention fwd Mqueries\u00b7heads/s at n=131k; % of BF16 tensor/H
 UNIT = "Mqueries\u00b7heads/s"
 
 
+def approx_error(Qf, Kf, Vf, Of, causal: bool, nrows: int = 256, seed: int = 7):
+    """Relative L2 error of the forward output against exact softmax attention, on seeded query rows of one
+    head: float64 numpy, straight from the definition softmax(q K^T) V (causal: keys up to the query)."""
+    n = Qf.shape[0]
+    rows = np.sort(np.random.default_rng(seed).choice(n, size=min(nrows, n), replace=False))
+    exact = np.empty((len(rows), Vf.shape[1]))
+    for i0 in range(0, len(rows), 32):
+        rr = rows[i0:i0 + 32]
+        s = Qf[rr] @ Kf.T
+        if causal:
+            s[np.arange(n)[None, :] > rr[:, None]] = -np.inf
+        s -= s.max(axis=1, keepdims=True)
+        p = np.exp(s)
+        exact[i0:i0 + 32] = (p @ Vf) / p.sum(axis=1, keepdims=True)
+    diff = Of[rows] - exact
+    per_row = np.linalg.norm(diff, axis=1) / np.linalg.norm(exact, axis=1)
+    return {"rel_l2": float(np.linalg.norm(diff) / np.linalg.norm(exact)), "median_row_rel_l2": float(np.median(per_row)),
+            "rows": int(len(rows)), "head": 0, "vs": "exact softmax attention (float64 numpy, sampled rows)"}
+
+
 def config_of(w: wl.Workload):
     return {"workload": w.name, "batch": w.batch, "heads": w.heads, "n": w.n, "d": w.d, "block": w.block, "m": w.m,
             "r": w.r, "causal": w.causal, "causal_base": w.base if w.causal else None, "input_dtype": w.dtype,
@@ -329,6 +349,11 @@ def run_ours(args, w: wl.Workload):
         if os.path.exists(src) and hashlib.sha256(open(src, "rb").read()).hexdigest() == tr["sha256"]:
             traffic = tr["bytes"]
 
+    err = None
+    if rank == 0:
+        f64 = lambda t: t.float().numpy().astype(np.float64)
+        err = approx_error(f64(hQ[0]), f64(hK[0]), f64(hV[0]), f64(hO[0]), w.causal)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         heads = list(range(min(args.cpu_heads, w.bh)))
@@ -352,6 +377,7 @@ def run_ours(args, w: wl.Workload):
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk.summary(),
             "cpu_baseline": cpu,
+            "approx_error": err,
         }
         print(json.dumps(line), flush=True)
     ha.close()

@@ -52,12 +52,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Wait until the phase with parity `parity` of the barrier has completed. Gives up (returns false) when
-// `*abort` becomes non-zero or after `limit_ns` of global time, in which case it sets `*abort` so that the
-// other warps of the CTA give up too.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort,
-                                          uint64_t limit_ns = 2000000000ull) {
-    if (mbar_try_wait(bar, parity)) return true;
+// Slow path of mbar_wait: polls with a bound in global time (kept out of line so that the timer read stays off
+// the fast path).
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int *abort, uint64_t limit_ns) {
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
@@ -69,6 +66,15 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
             }
         }
     }
+}
+
+// Wait until the phase with parity `parity` of the barrier has completed. Gives up (returns false) when
+// `*abort` becomes non-zero or after `limit_ns` of global time, in which case it sets `*abort` so that the
+// other warps of the CTA give up too.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort,
+                                          uint64_t limit_ns = 2000000000ull) {
+    if (__builtin_expect(mbar_try_wait(bar, parity), 1)) return true;
+    return mbar_wait_slow(bar, parity, abort, limit_ns);
 }
 
 // --------------------------------------------------------------------------------------------- TMA

@@ -160,8 +160,15 @@ template <int D>
 struct Cfg {
     static constexpr int R = D == 64 ? 3 : 2;          // S ring buffers
     static constexpr int QB = D == 64 ? 2 : 1;         // Q buffers per tile
-    static constexpr int NST = D == 64 ? 3 : 2;        // K/V stages
+    static constexpr int NST = D == 64 ? 4 : 2;        // K/V stages
+    // P.V products issued per group before the score products that reuse their buffers: two keep a score
+    // product from queueing right behind the P.V that reads its buffer (a tensor-pipe stall; d = 128 is bound
+    // by the pipe), one gives the second tile its next score tile sooner (d = 64 is bound by the softmax)
+    static constexpr int kGroup = D == 64 ? 1 : 2;
     static constexpr int SEG = D == 64 ? 128 : 64;     // bytes per row segment of the staged output stores
+    // d = 64: the epilogue stages its output rows in the item's own Q buffer (dead once the tile's last score
+    // product has completed; the Q loader refills it only after the epilogue); d = 128 has a stage of its own
+    static constexpr bool kStageInQ = D == 64;
     static constexpr int kOCol = R * 128;              // first O column
     static constexpr int kTileBytes = 128 * D * 2;     // 128 rows of bf16 (a Q tile, a K or a V chunk)
     static constexpr int kQ = 0;
@@ -175,17 +182,18 @@ struct Cfg {
     static constexpr int kRows = kQPerm + 128 * 4;                         // global rows of each stage
     static constexpr int kWord = kRows + NST * 128 * 4;
     static constexpr int kStage = (kWord + NST * 4 + 64 + 15) / 16 * 16;   // 8 softmax warps x 32 rows x SEG
-    static constexpr int kBars = kStage + 8 * 32 * SEG;
+    static constexpr int kBars = kStage + (kStageInQ ? 0 : 8 * 32 * SEG);
     static constexpr int bQFull = 0, bQEmpty = bQFull + 2 * QB, bKVFull = bQEmpty + 2 * QB,
                          bKVEmpty = bKVFull + NST, bWordFull = bKVEmpty + NST, bRowsFull = bWordFull + NST,
                          bSFull = bRowsFull + NST,
                          bPFull = bSFull + R, bOReady = bPFull + R, bOFinal = bOReady + 4, bOFree = bOFinal + 2,
-                         bDrain = bOFree + 2, kNumBars = bDrain + 1;
+                         bDrain = bOFree + 2, bQStage = bDrain + 1, kNumBars = bQStage + 2 * QB;
     static constexpr int kTmemSlot = kBars + kNumBars * 8;
     static constexpr int kAbort = kTmemSlot + 4;
     static constexpr int kBytes = kAbort + 4;
     static_assert(kBars % 8 == 0, "mbarriers need 8-byte alignment");
     static_assert(kStage % 16 == 0, "16-byte stage pieces");
+    static_assert(!kStageInQ || 4 * 32 * SEG <= kTileBytes, "a tile's four warps stage in its Q buffer");
     static_assert(kBytes + 1024 <= 232448, "shared memory budget");
     static_assert(kOCol + 2 * D <= 512, "TMEM budget");
 };
@@ -278,6 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
         for (int i = 0; i < 2 * C::QB; ++i) {
             mbar_init(bar(C::bQFull + i), 32);     // the Q loader's lanes (copy completion)
             mbar_init(bar(C::bQEmpty + i), 1);
+            mbar_init(bar(C::bQStage + i), 128);   // the tile's softmax threads, after an epilogue staged there
         }
         for (int s = 0; s < C::NST; ++s) {
             mbar_init(bar(C::bKVFull + s), 64);    // the K and V loader warps' lanes (copy completion)
@@ -339,6 +348,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                 const int qb = qc % C::QB;
                 const int use = qc / C::QB;
                 if (use > 0 && !mbar_wait(bar(C::bQEmpty + t * C::QB + qb), (use - 1) & 1, abort_flag)) {
+                    ok = false;
+                    continue;
+                }
+                if (C::kStageInQ && use > 0 && !mbar_wait(bar(C::bQStage + t * C::QB + qb), (use - 1) & 1, abort_flag)) {
                     ok = false;
                     continue;
                 }
@@ -587,21 +600,26 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                     // the chunk's stage is free once every tile that uses it has issued its P.V
                     const bool last_user = t == 1 || c >= x.nc1;
                     if (last_user) mma_commit(bar(C::bKVEmpty + slot));
-                    // the ring buffer of pair k is free again: fill it with the score tile R pairs ahead
-                    const int ka = k + C::R;
-                    if (ka < np) {
-                        ok = issue_s(cur, ka);
-                    } else if (look) {
-                        const int kn = ka - np;
-                        if (kn == nxt.pre && kn < nxt.x.npairs) {
-                            int tn, cn;
-                            pair_tc(nxt.x, kn, tn, cn);
-                            // with one Q buffer per tile, the next Q is loaded only after this item's last S:
-                            // take it only if it is already there
-                            if (get_q(nxt, tn, C::QB > 1)) ok = issue_s(nxt, kn);
-                            else look = false;
-                        } else {
-                            look = false;
+                    // the ring buffers of this pair group (kGroup = 2: pairs k-1 and k, or k alone at an odd end) are
+                    // free again: fill them with the score tiles R pairs ahead
+                    if (C::kGroup == 1 || (k & 1) || k == np - 1) {
+                        for (int kg = (C::kGroup == 2 && (k & 1)) ? k - 1 : k; kg <= k && ok; ++kg) {
+                            const int ka = kg + C::R;
+                            if (ka < np) {
+                                ok = issue_s(cur, ka);
+                            } else if (look) {
+                                const int kn = ka - np;
+                                if (kn == nxt.pre && kn < nxt.x.npairs) {
+                                    int tn, cn;
+                                    pair_tc(nxt.x, kn, tn, cn);
+                                    // with one Q buffer per tile, the next Q is loaded only after this item's last S:
+                                    // take it only if it is already there
+                                    if (get_q(nxt, tn, C::QB > 1)) ok = issue_s(nxt, kn);
+                                    else look = false;
+                                } else {
+                                    look = false;
+                                }
+                            }
                         }
                     }
                 }
@@ -624,6 +642,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
         const uint32_t tO = trow + C::kOCol + t * D;
         uint32_t kp = 0, g = 0;
         int hp0 = 0, hp1 = 0, fin = 0;               // P handoffs per chunk parity; epilogues done
+        int qn = 0;                                  // items of this tile so far (its Q buffer is qn mod QB)
         bool ok = true;
         for (int64_t it = first; it < last && ok; it += stride) {
             const Item x = decode(a, it);
@@ -750,7 +769,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
             tc_fence_after();
             const float inv_l = 1.0f / l;
             const float Lrow = (m_run + __log2f(l)) * kLn2;   // natural log of the row's normaliser
-            unsigned char *stage = sm + C::kStage + (warp - 4) * (32 * C::SEG);
+            const int qbuf = t * C::QB + qn % C::QB;
+            unsigned char *stage = C::kStageInQ ? sm + C::kQ + qbuf * C::kTileBytes + q * (32 * C::SEG)
+                                                : sm + C::kStage + (warp - 4) * (32 * C::SEG);
             auto o_scaled = [&](float scale) {
                 return [&, scale](int j, float (&v)[32]) {
                     uint32_t o[32];
@@ -826,6 +847,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                 unsigned char *drow = static_cast<unsigned char *>(a.O) + orow * D * esz;
                 warp_write_rows<D, C::SEG>(stage, drow, a.out_dtype == 0, lane, merged);
             }
+            if (C::kStageInQ) {
+                // the stage writes are ordered before the tensor core's later reads of the refilled buffer
+                fence_proxy_async_smem();
+                mbar_arrive(bar(C::bQStage + qbuf));   // the Q buffer may be refilled
+            }
+            ++qn;
             tc_fence_before();
             mbar_arrive(bar(C::bOFree + t));
             kp += x.npairs;

@@ -9,8 +9,8 @@
 // chains over k = 0..d-1 from +0, so the sign decision is reproducible bit for bit. A row whose smallest
 // |x.P_j| is below 1e-4 * ||x||_2 is flagged as near zero.
 //
-// Layout: persistent CTAs of 128 threads walk tiles of 128 consecutive rows of the combined index
-// g = ((bh*2 + which)*n + row) (which 0 = Q, 1 = K), one row per thread. Tiles are double-buffered in
+// Layout: persistent CTAs of 128 threads walk tiles of 128 x RPT consecutive rows of the combined index
+// g = ((bh*2 + which)*n + row) (which 0 = Q, 1 = K), RPT rows per thread. Tiles are double-buffered in
 // shared memory: the 16-byte cp.async copies of tile i+1 (coalesced; row stride padded by 16 bytes against
 // bank conflicts) are in flight while tile i is hashed. P sits in shared memory as [d][r4] (r rounded up to
 // a multiple of 4); for each k a thread reads P[k][0..r) with broadcast 16-byte loads and advances each
@@ -21,12 +21,15 @@
 namespace ha {
 namespace {
 
-constexpr int kRows = 128;
+constexpr int kThreads = 128;
 
-template <int D, int DTYPE, int R4>
-__global__ void __launch_bounds__(kRows) hash_kernel(const void *__restrict__ Q, const void *__restrict__ K,
-                                                     int64_t n, int64_t total_rows, const float *__restrict__ P,
-                                                     int r, uint16_t *__restrict__ rank, uint8_t *__restrict__ near) {
+// RPT rows per thread: a tile is kThreads * RPT consecutive rows; thread i hashes rows i, i + kThreads, ...
+// Each broadcast load of P then feeds RPT rows' fused multiply-adds.
+template <int D, int DTYPE, int R4, int RPT>
+__global__ void __launch_bounds__(kThreads) hash_kernel(const void *__restrict__ Q, const void *__restrict__ K,
+                                                        int64_t n, int64_t total_rows, const float *__restrict__ P,
+                                                        int r, uint16_t *__restrict__ rank, uint8_t *__restrict__ near) {
+    constexpr int kRows = kThreads * RPT;
     constexpr int ESZ = DTYPE == 0 ? 2 : 4;
     constexpr int ROW_BYTES = D * ESZ;
     constexpr int STRIDE = ROW_BYTES + 16;
@@ -40,27 +43,37 @@ __global__ void __launch_bounds__(kRows) hash_kernel(const void *__restrict__ Q,
     unsigned char *tiles = smem + D * PS * sizeof(float);                      // [2][kRows][STRIDE]
 
     const int tid = threadIdx.x;
-    for (int i = tid; i < D * PS; i += kRows) {
+    for (int i = tid; i < D * PS; i += kThreads) {
         const int k = i / PS, j = i % PS;
         Ps[i] = j < r ? P[k * r + j] : 0.0f;
     }
     const int64_t ntiles = (total_rows + kRows - 1) / kRows;
 
-    // stage one tile: 16-byte pieces, CHUNKS consecutive threads per row. The tile's first row is located
-    // once (segment = g / n); later rows step forward, wrapping into the next segment at most 128 / n times.
+    // stage one tile with 16-byte copies. A tile inside one segment (the usual case) is kRows * ROW_BYTES
+    // contiguous bytes; a tile that straddles segments locates each row (segment = g / n).
     auto stage = [&](int64_t tile, int buf) {
         unsigned char *dst = tiles + buf * (kRows * STRIDE);
         const int64_t g0 = tile * kRows;
         const int64_t seg0 = g0 / n, rr0 = g0 - seg0 * n;
-        const int ch = tid % CHUNKS;
-        for (int row = tid / CHUNKS; row < kRows; row += kRows / CHUNKS) {
-            if (g0 + row >= total_rows) break;
-            int64_t seg = seg0, rr = rr0 + row;
-            while (rr >= n) { rr -= n; ++seg; }
-            const int64_t which = seg & 1, bhi = seg >> 1;
-            const unsigned char *src = static_cast<const unsigned char *>(which ? K : Q) +
-                                       ((bhi * n + rr) * D) * ESZ + ch * 16;
-            cp_async_16(dst + row * STRIDE + ch * 16, src);
+        if (rr0 + kRows <= n) {
+            const unsigned char *src = static_cast<const unsigned char *>((seg0 & 1) ? K : Q) +
+                                       ((seg0 >> 1) * n + rr0) * ROW_BYTES;
+#pragma unroll 4
+            for (int i = tid; i < kRows * CHUNKS; i += kThreads) {
+                const int row = i / CHUNKS, ch = i % CHUNKS;
+                cp_async_16(dst + row * STRIDE + ch * 16, src + static_cast<int64_t>(i) * 16);
+            }
+        } else {
+            const int ch = tid % CHUNKS;
+            for (int row = tid / CHUNKS; row < kRows; row += kThreads / CHUNKS) {
+                if (g0 + row >= total_rows) break;
+                int64_t seg = seg0, rr = rr0 + row;
+                while (rr >= n) { rr -= n; ++seg; }
+                const int64_t which = seg & 1, bhi = seg >> 1;
+                const unsigned char *src = static_cast<const unsigned char *>(which ? K : Q) +
+                                           ((bhi * n + rr) * D) * ESZ + ch * 16;
+                cp_async_16(dst + row * STRIDE + ch * 16, src);
+            }
         }
         cp_async_commit();
     };
@@ -78,53 +91,66 @@ __global__ void __launch_bounds__(kRows) hash_kernel(const void *__restrict__ Q,
         }
         __syncthreads();   // tile `buf` (and P on the first pass) visible to every thread
 
-        const int64_t g = tile * kRows + tid;
-        if (g < total_rows) {
-            const unsigned char *row = tiles + buf * (kRows * STRIDE) + tid * STRIDE;
-            float acc[R4 > 0 ? R4 : 1];
+        const unsigned char *rows = tiles + buf * (kRows * STRIDE) + tid * STRIDE;
+        float acc[RPT][R4 > 0 ? R4 : 1];
+        float nrm2[RPT];
 #pragma unroll
-            for (int j = 0; j < R4; ++j) acc[j] = 0.0f;
-            float nrm2 = 0.0f;
+        for (int q = 0; q < RPT; ++q) {
+            nrm2[q] = 0.0f;
+#pragma unroll
+            for (int j = 0; j < R4; ++j) acc[q][j] = 0.0f;
+        }
 #pragma unroll 2
-            for (int c = 0; c < CHUNKS; ++c) {
-                const uint4 v = *reinterpret_cast<const uint4 *>(row + c * 16);
-                float x[EPC];
+        for (int c = 0; c < CHUNKS; ++c) {
+            float x[RPT][EPC];
+#pragma unroll
+            for (int q = 0; q < RPT; ++q) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(rows + q * (kThreads * STRIDE) + c * 16);
                 if (DTYPE == 0) {
                     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        x[2 * e] = __uint_as_float(w[e] << 16);
-                        x[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+                        x[q][2 * e] = __uint_as_float(w[e] << 16);
+                        x[q][2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
                     }
                 } else {
-                    x[0] = __uint_as_float(v.x);
-                    x[1] = __uint_as_float(v.y);
-                    x[2] = __uint_as_float(v.z);
-                    x[3] = __uint_as_float(v.w);
+                    x[q][0] = __uint_as_float(v.x);
+                    x[q][1] = __uint_as_float(v.y);
+                    x[q][2] = __uint_as_float(v.z);
+                    x[q][3] = __uint_as_float(v.w);
                 }
+            }
 #pragma unroll
-                for (int e = 0; e < EPC; ++e) {
-                    const int k = c * EPC + e;
-                    nrm2 = __fmaf_rn(x[e], x[e], nrm2);
-                    const float4 *pk = reinterpret_cast<const float4 *>(Ps + k * PS);
+            for (int e = 0; e < EPC; ++e) {
+                const int k = c * EPC + e;
 #pragma unroll
-                    for (int q4 = 0; q4 < R4 / 4; ++q4) {
-                        const float4 p = pk[q4];
-                        acc[4 * q4 + 0] = __fmaf_rn(x[e], p.x, acc[4 * q4 + 0]);
-                        acc[4 * q4 + 1] = __fmaf_rn(x[e], p.y, acc[4 * q4 + 1]);
-                        acc[4 * q4 + 2] = __fmaf_rn(x[e], p.z, acc[4 * q4 + 2]);
-                        acc[4 * q4 + 3] = __fmaf_rn(x[e], p.w, acc[4 * q4 + 3]);
+                for (int q = 0; q < RPT; ++q) nrm2[q] = __fmaf_rn(x[q][e], x[q][e], nrm2[q]);
+                const float4 *pk = reinterpret_cast<const float4 *>(Ps + k * PS);
+#pragma unroll
+                for (int q4 = 0; q4 < R4 / 4; ++q4) {
+                    const float4 p = pk[q4];
+#pragma unroll
+                    for (int q = 0; q < RPT; ++q) {
+                        acc[q][4 * q4 + 0] = __fmaf_rn(x[q][e], p.x, acc[q][4 * q4 + 0]);
+                        acc[q][4 * q4 + 1] = __fmaf_rn(x[q][e], p.y, acc[q][4 * q4 + 1]);
+                        acc[q][4 * q4 + 2] = __fmaf_rn(x[q][e], p.z, acc[q][4 * q4 + 2]);
+                        acc[q][4 * q4 + 3] = __fmaf_rn(x[q][e], p.w, acc[q][4 * q4 + 3]);
                     }
                 }
             }
-            const float thr = __fmul_rn(1e-4f, __fsqrt_rn(nrm2));
+        }
+#pragma unroll
+        for (int q = 0; q < RPT; ++q) {
+            const int64_t g = tile * kRows + q * kThreads + tid;
+            if (g >= total_rows) continue;
+            const float thr = __fmul_rn(1e-4f, __fsqrt_rn(nrm2[q]));
             uint32_t code = 0;
             bool flag = false;
 #pragma unroll
             for (int j = 0; j < R4; ++j) {
                 if (j < r) {
-                    code |= (acc[j] > 0.0f ? 1u : 0u) << j;
-                    flag |= fabsf(acc[j]) < thr;
+                    code |= (acc[q][j] > 0.0f ? 1u : 0u) << j;
+                    flag |= fabsf(acc[q][j]) < thr;
                 }
             }
             // inverse Gray code: prefix XOR of all right shifts (16-bit codes)
@@ -150,18 +176,21 @@ template <int D, int DTYPE, int R4>
 int launch_hash_t(const void *Q, const void *K, int64_t bh, int64_t n, const float *P, int r, uint16_t *rank,
                   uint8_t *near, cudaStream_t st) {
     constexpr int ESZ = DTYPE == 0 ? 2 : 4;
+    // two rows per thread while a double-buffered tile stays small (rows of up to 256 bytes)
+    constexpr int RPT = D * ESZ <= 256 ? 2 : 1;
+    constexpr int kRows = kThreads * RPT;
     const size_t smem = D * (R4 > 0 ? R4 : 4) * sizeof(float) + 2 * kRows * (D * ESZ + 16);
-    auto kern = hash_kernel<D, DTYPE, R4>;
+    auto kern = hash_kernel<D, DTYPE, R4, RPT>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
         return -1;
     int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kRows, smem) != cudaSuccess || per_sm < 1)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem) != cudaSuccess || per_sm < 1)
         per_sm = 1;
     const int64_t total = 2 * bh * n;
     const int64_t ntiles = (total + kRows - 1) / kRows;
     const int64_t slots = static_cast<int64_t>(num_sms_hash()) * per_sm;
     const int64_t grid = ntiles < slots ? ntiles : slots;
-    kern<<<static_cast<unsigned>(grid), kRows, smem, st>>>(Q, K, n, total, P, r, rank, near);
+    kern<<<static_cast<unsigned>(grid), kThreads, smem, st>>>(Q, K, n, total, P, r, rank, near);
     return cudaPeekAtLastError() == cudaSuccess ? 1 : -1;
 }
 

@@ -12,7 +12,8 @@
 //              (chunk, digit) pair (digit-major, chunks in order);
 //   scatter -- per chunk, 8 warps each own a contiguous 256-row slice; a warp ranks equal digits inside a
 //              32-row step with __match_any_sync and keeps running per-digit counters, so rows leave in
-//              their original order within each digit.
+//              their original order within each digit. The chunk is ordered in shared memory first, so
+//              that the permutation is written in runs of consecutive slots.
 // No kernel waits on another CTA: the three launches replace a look-back scan.
 #include "ha_common.cuh"
 #include "ha_internal.h"
@@ -66,12 +67,19 @@ __global__ void __launch_bounds__(1024) sort_scan_kernel(int radix, int cps, int
     __shared__ int tot[1 << kMaxPassBits];
     const int64_t s = blockIdx.x;
     int32_t *h = hist + s * cps * radix;
+    // the chunk counts of a digit are read 16 at a time, so that the loads are in flight together
+    constexpr int U = 16;
     for (int b = threadIdx.x; b < radix; b += blockDim.x) {
         int run = 0;
-        for (int c = 0; c < cps; ++c) {
-            const int t = h[c * radix + b];
-            h[c * radix + b] = run;
-            run += t;
+        for (int c0 = 0; c0 < cps; c0 += U) {
+            int t[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) t[u] = c0 + u < cps ? h[(c0 + u) * radix + b] : 0;
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (c0 + u < cps) h[(c0 + u) * radix + b] = run;
+                run += t[u];
+            }
         }
         tot[b] = run;
     }
@@ -86,21 +94,78 @@ __global__ void __launch_bounds__(1024) sort_scan_kernel(int radix, int cps, int
     }
     if (b < radix) {
         const int base = b == 0 ? 0 : tot[b - 1];
-        for (int c = 0; c < cps; ++c) h[c * radix + b] += base;
+        for (int c0 = 0; c0 < cps; c0 += U) {
+            int t[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) t[u] = c0 + u < cps ? h[(c0 + u) * radix + b] : 0;
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+                if (c0 + u < cps) h[(c0 + u) * radix + b] = t[u] + base;
+        }
     }
 }
 
+// Exclusive prefix sum of a[0..R) in place by a block of kSortWarps * 32 threads (R <= 4 * blockDim).
+__device__ __forceinline__ void block_exclusive_scan(int *a, int R, int *warp_sums) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int per = (R + blockDim.x - 1) / blockDim.x;
+    const int b0 = threadIdx.x * per;
+    int v[4];
+    int sum = 0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        v[u] = (u < per && b0 + u < R) ? a[b0 + u] : 0;
+        sum += v[u];
+    }
+    int x = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, off);
+        if (lane >= off) x += y;
+    }
+    if (lane == 31) warp_sums[warp] = x;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int run = 0;
+        for (int w = 0; w < kSortWarps; ++w) {
+            const int t = warp_sums[w];
+            warp_sums[w] = run;
+            run += t;
+        }
+    }
+    __syncthreads();
+    int run = warp_sums[warp] + x - sum;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        if (u < per && b0 + u < R) a[b0 + u] = run;
+        run += v[u];
+    }
+    __syncthreads();
+}
+
+// Per chunk: rank the rows stably by digit (warps own contiguous 256-row slices; within a 32-row step equal
+// digits are ranked with __match_any_sync), giving each row its local position in the chunk's digit-sorted
+// order and its global position (the digit's first slot for this chunk, from the scan, plus its rank among
+// the chunk's rows of that digit). The inverse permutation is written in row order; the permutation is
+// written from the digit-sorted order, so that rows of one digit land in consecutive slots.
 __global__ void __launch_bounds__(kSortWarps * 32) sort_scatter_kernel(Level lv, const uint16_t *__restrict__ rank,
                                                                        SortPass ps, const int32_t *__restrict__ in_idx,
                                                                        const int32_t *__restrict__ hist, int cps,
                                                                        int32_t *__restrict__ perm,
                                                                        int32_t *__restrict__ inv) {
-    extern __shared__ int wcnt[];   // [kSortWarps][radix]
+    extern __shared__ int sm[];
+    const int R = ps.radix;
+    int *wcnt = sm;                               // [kSortWarps][R]: per-warp digit counts, then local offsets
+    int *coff = wcnt + kSortWarps * R;            // [R]: first local position of each digit in the chunk
+    int *gbase = coff + R;                        // [R]: first global position of each digit for this chunk
+    int *wsum = gbase + R;                        // [kSortWarps]
+    int32_t *srow = wsum + kSortWarps;            // [kSortChunk]: rows in local (digit-sorted) order
+    int32_t *sgpos = srow + kSortChunk;           // [kSortChunk]: their global positions
     const int64_t s = blockIdx.x / cps;
     const int c = blockIdx.x % cps;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const unsigned lt_mask = (1u << lane) - 1u;
-    for (int i = threadIdx.x; i < kSortWarps * ps.radix; i += blockDim.x) wcnt[i] = 0;
+    for (int i = threadIdx.x; i < kSortWarps * R; i += blockDim.x) wcnt[i] = 0;
     __syncthreads();
 
     const SegView v = seg_view(lv, rank, s);
@@ -109,7 +174,7 @@ __global__ void __launch_bounds__(kSortWarps * 32) sort_scatter_kernel(Level lv,
     constexpr int kSlice = kSortChunk / kSortWarps;
     const int64_t lo = min(end, start + static_cast<int64_t>(warp) * kSlice);
     const int64_t hi = min(end, lo + kSlice);
-    int *mycnt = wcnt + warp * ps.radix;
+    int *mycnt = wcnt + warp * R;
 
     for (int64_t base = lo; base < hi; base += 32) {
         const int64_t p = base + lane;
@@ -120,12 +185,20 @@ __global__ void __launch_bounds__(kSortWarps * 32) sort_scatter_kernel(Level lv,
         if (valid && lane == __ffs(peers) - 1) mycnt[key] += __popc(peers);
     }
     __syncthreads();
-    const int32_t *h = hist + (s * cps + c) * ps.radix;
-    for (int b = threadIdx.x; b < ps.radix; b += blockDim.x) {
-        int run = h[b];
+    const int32_t *h = hist + (s * cps + c) * R;
+    for (int b = threadIdx.x; b < R; b += blockDim.x) {
+        int tot = 0;
+        for (int w = 0; w < kSortWarps; ++w) tot += wcnt[w * R + b];
+        coff[b] = tot;
+        gbase[b] = h[b];
+    }
+    __syncthreads();
+    block_exclusive_scan(coff, R, wsum);
+    for (int b = threadIdx.x; b < R; b += blockDim.x) {
+        int run = coff[b];
         for (int w = 0; w < kSortWarps; ++w) {
-            const int t = wcnt[w * ps.radix + b];
-            wcnt[w * ps.radix + b] = run;
+            const int t = wcnt[w * R + b];
+            wcnt[w * R + b] = run;
             run += t;
         }
     }
@@ -141,11 +214,16 @@ __global__ void __launch_bounds__(kSortWarps * 32) sort_scatter_kernel(Level lv,
         if (valid && lane == __ffs(peers) - 1) mycnt[key] = first + __popc(peers);
         __syncwarp();
         if (valid) {
-            const int pos = first + __popc(peers & lt_mask);
-            perm[v.out + pos] = row;
-            if (inv) inv[v.out + row] = pos;
+            const int lpos = first + __popc(peers & lt_mask);
+            const int gpos = gbase[key] + (lpos - coff[key]);
+            if (inv) inv[v.out + row] = gpos;
+            srow[lpos] = row;
+            sgpos[lpos] = gpos;
         }
     }
+    __syncthreads();
+    const int nloc = static_cast<int>(end - start);
+    for (int lp = threadIdx.x; lp < nloc; lp += blockDim.x) perm[v.out + sgpos[lp]] = srow[lp];
 }
 
 }  // namespace
@@ -158,7 +236,11 @@ int launch_sort_pass(const Level &lv, const uint16_t *rank, SortPass ps, const i
     const int64_t grid = nseg * cps;
     sort_count_kernel<<<static_cast<unsigned>(grid), 256, ps.radix * sizeof(int), st>>>(lv, rank, ps, in_idx, hist, cps);
     sort_scan_kernel<<<static_cast<unsigned>(nseg), 1024, 0, st>>>(ps.radix, cps, hist);
-    const size_t smem = static_cast<size_t>(kSortWarps) * ps.radix * sizeof(int);
+    const size_t smem = (static_cast<size_t>(kSortWarps + 2) * ps.radix + kSortWarps + 2 * kSortChunk) * sizeof(int);
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(sort_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+            cudaSuccess)
+        return -1;
     sort_scatter_kernel<<<static_cast<unsigned>(grid), kSortWarps * 32, smem, st>>>(lv, rank, ps, in_idx, hist, cps,
                                                                                     perm, inv);
     return cudaPeekAtLastError() == cudaSuccess ? 3 : -1;

@@ -176,13 +176,26 @@ __global__ void __launch_bounds__(kSortWarps * 32) sort_scatter_kernel(Level lv,
     const int64_t hi = min(end, lo + kSlice);
     int *mycnt = wcnt + warp * R;
 
-    for (int64_t base = lo; base < hi; base += 32) {
-        const int64_t p = base + lane;
-        const bool valid = p < hi;
-        int32_t row = 0;
-        const int key = valid ? digit_of(v, in_idx, p, ps, row) : -1;
+    // one ranking pass: the slice's digits (loads issued together), each row's rank among the earlier rows of
+    // its digit in the slice (kept in registers), and the slice's per-digit counts
+    constexpr int STEPS = kSlice / 32;
+    int keyv[STEPS], rk[STEPS];
+    int32_t rowv[STEPS];
+#pragma unroll
+    for (int i = 0; i < STEPS; ++i) {
+        const int64_t p = lo + i * 32 + lane;
+        rowv[i] = 0;
+        keyv[i] = p < hi ? digit_of(v, in_idx, p, ps, rowv[i]) : -1;
+    }
+#pragma unroll
+    for (int i = 0; i < STEPS; ++i) {
+        const int key = keyv[i];
         const unsigned peers = __match_any_sync(0xffffffffu, key);
-        if (valid && lane == __ffs(peers) - 1) mycnt[key] += __popc(peers);
+        const int before = key >= 0 ? mycnt[key] : 0;
+        __syncwarp();
+        if (key >= 0 && lane == __ffs(peers) - 1) mycnt[key] = before + __popc(peers);
+        __syncwarp();
+        rk[i] = before + __popc(peers & lt_mask);
     }
     __syncthreads();
     const int32_t *h = hist + (s * cps + c) * R;
@@ -203,21 +216,14 @@ __global__ void __launch_bounds__(kSortWarps * 32) sort_scatter_kernel(Level lv,
         }
     }
     __syncthreads();
-    for (int64_t base = lo; base < hi; base += 32) {
-        const int64_t p = base + lane;
-        const bool valid = p < hi;
-        int32_t row = 0;
-        const int key = valid ? digit_of(v, in_idx, p, ps, row) : -1;
-        const unsigned peers = __match_any_sync(0xffffffffu, key);
-        const int first = valid ? mycnt[key] : 0;
-        __syncwarp();
-        if (valid && lane == __ffs(peers) - 1) mycnt[key] = first + __popc(peers);
-        __syncwarp();
-        if (valid) {
-            const int lpos = first + __popc(peers & lt_mask);
+#pragma unroll
+    for (int i = 0; i < STEPS; ++i) {
+        const int key = keyv[i];
+        if (key >= 0) {
+            const int lpos = mycnt[key] + rk[i];
             const int gpos = gbase[key] + (lpos - coff[key]);
-            if (inv) inv[v.out + row] = gpos;
-            srow[lpos] = row;
+            if (inv) inv[v.out + rowv[i]] = gpos;
+            srow[lpos] = rowv[i];
             sgpos[lpos] = gpos;
         }
     }

@@ -21,9 +21,11 @@ struct hyper_attn_s {
     unsigned char *pin = nullptr;
     size_t pin_bytes = 0;
     cudaEvent_t pin_free = nullptr;
-    // device copies for hyper_attn_forward_host (grow-only)
+    // device copies for hyper_attn_forward_host (grow-only), and its copy streams and chunk events
     unsigned char *io = nullptr;
     size_t io_bytes = 0;
+    cudaStream_t cs_in = nullptr, cs_out = nullptr;
+    std::vector<cudaEvent_t> pipe_ev;
     // draws currently resident in the workspace
     bool draws_valid = false;
     uint64_t dk_seed = 0;
@@ -273,9 +275,9 @@ int host_draws(uint64_t seed, const Shape &s, int64_t bh_offset, float *P, int32
     return 0;
 }
 
-int upload_draws(hyper_attn_t h, uint64_t seed, const Shape &s, cudaStream_t st) {
+int upload_draws(hyper_attn_t h, uint64_t seed, const Shape &s, int64_t bh_offset, cudaStream_t st) {
     if (h->draws_valid && h->dk_seed == seed && h->dk_d == s.d && h->dk_r == s.r && h->dk_m == s.m &&
-        h->dk_causal == s.causal && h->dk_bh == s.bh && h->dk_n == s.n && h->dk_off == h->opt.bh_offset &&
+        h->dk_causal == s.causal && h->dk_bh == s.bh && h->dk_n == s.n && h->dk_off == bh_offset &&
         (!s.causal || h->dk_base == h->opt.causal_base))
         return HA_OK;
     const size_t pbytes = sizeof(float) * ha::kMaxR * 128;
@@ -285,18 +287,19 @@ int upload_draws(hyper_attn_t h, uint64_t seed, const Shape &s, cudaStream_t st)
     HA_CUDA(h, cudaEventSynchronize(h->pin_free));   // the previous upload has left the staging buffer
     float *P = reinterpret_cast<float *>(h->pin);
     int32_t *S = reinterpret_cast<int32_t *>(h->pin + pbytes);
-    if (host_draws(seed, s, h->opt.bh_offset, P, S)) return fail(h, HA_ERR_INVALID_ARG, "sample draw failed");
+    if (host_draws(seed, s, bh_offset, P, S)) return fail(h, HA_ERR_INVALID_ARG, "sample draw failed");
     HA_CUDA(h, cudaMemcpyAsync(h->ws + h->lay.P, P, sizeof(float) * s.d * (s.r ? s.r : 1), cudaMemcpyHostToDevice, st));
     if (sbytes) HA_CUDA(h, cudaMemcpyAsync(h->ws + h->lay.S, S, sbytes, cudaMemcpyHostToDevice, st));
     HA_CUDA(h, cudaEventRecord(h->pin_free, st));
     h->draws_valid = true;
     h->dk_seed = seed; h->dk_d = s.d; h->dk_r = s.r; h->dk_m = s.m; h->dk_causal = s.causal;
-    h->dk_bh = s.bh; h->dk_n = s.n; h->dk_base = h->opt.causal_base; h->dk_off = h->opt.bh_offset;
+    h->dk_bh = s.bh; h->dk_n = s.n; h->dk_base = h->opt.causal_base; h->dk_off = bh_offset;
     return HA_OK;
 }
 
+// The forward pass of shape s on device buffers; the problems' draws are keyed from global index bh_offset.
 int run_forward(hyper_attn_t h, const void *Q, const void *K, const void *V, void *O, const Shape &s,
-                uint64_t seed) {
+                uint64_t seed, int64_t bh_offset) {
     cudaStream_t st = static_cast<cudaStream_t>(h->opt.stream);
     const int dtype = h->opt.dtype;
     const int out_dtype = h->opt.out_dtype < 0 ? dtype : h->opt.out_dtype;
@@ -317,7 +320,7 @@ int run_forward(hyper_attn_t h, const void *Q, const void *K, const void *V, voi
     if (h->have_last && (lay.P != h->lay.P || lay.S != h->lay.S)) h->draws_valid = false;
     h->lay = lay;
     h->have_last = true;
-    rc = upload_draws(h, seed, s, st);
+    rc = upload_draws(h, seed, s, bh_offset, st);
     if (rc) return rc;
 
     unsigned char *ws = h->ws;
@@ -509,7 +512,7 @@ int hyper_attn_forward(hyper_attn_t h, const void *Q, const void *K, const void 
     rc = check_shape(h, n, d, h->opt.batch * heads, block, m, r, causal, &s);
     if (rc) return rc;
     DeviceGuard g(h->device);
-    return run_forward(h, Q, K, V, O, s, seed);
+    return run_forward(h, Q, K, V, O, s, seed, h->opt.bh_offset);
 }
 
 int hyper_attn_forward_host(hyper_attn_t h, const void *Q, const void *K, const void *V, void *O, int64_t n, int d,
@@ -543,15 +546,58 @@ int hyper_attn_forward_host(hyper_attn_t h, const void *Q, const void *K, const 
     }
     unsigned char *dQ = h->io, *dK = dQ + align_up(in_bytes), *dV = dK + align_up(in_bytes);
     unsigned char *dO = dV + align_up(in_bytes);
-    HA_CUDA(h, cudaMemcpyAsync(dQ, Q, in_bytes, cudaMemcpyHostToDevice, st));
-    HA_CUDA(h, cudaMemcpyAsync(dK, K, in_bytes, cudaMemcpyHostToDevice, st));
-    HA_CUDA(h, cudaMemcpyAsync(dV, V, in_bytes, cudaMemcpyHostToDevice, st));
-    rc = run_forward(h, dQ, dK, dV, dO, s, seed);
+    // The problems are independent: they go through in up to kChunks contiguous groups, so that the copy of
+    // group i+1 to the device, the forward pass of group i (on the handle's stream) and the copy of group i-1's
+    // output back overlap (two copy streams; page-locked host buffers are needed for the overlap). Each group's
+    // draws are keyed from its global problem index, so the output equals one pass over all problems. With
+    // debug captures on, one group (the captures then describe the whole call).
+    constexpr int64_t kChunks = 8;
+    const int64_t nchunk = h->opt.debug_captures ? 1 : (s.bh < kChunks ? s.bh : kChunks);
+    if (!h->cs_in) {
+        HA_CUDA(h, cudaStreamCreateWithFlags(&h->cs_in, cudaStreamNonBlocking));
+        HA_CUDA(h, cudaStreamCreateWithFlags(&h->cs_out, cudaStreamNonBlocking));
+    }
+    while (h->pipe_ev.size() < static_cast<size_t>(2 * kChunks + 1)) {
+        cudaEvent_t e;
+        HA_CUDA(h, cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+        h->pipe_ev.push_back(e);
+    }
+    cudaEvent_t ev_start = h->pipe_ev[2 * kChunks];
+    HA_CUDA(h, cudaEventRecord(ev_start, st));   // earlier work on the handle's stream comes first
+    HA_CUDA(h, cudaStreamWaitEvent(h->cs_in, ev_start, 0));
+    HA_CUDA(h, cudaStreamWaitEvent(h->cs_out, ev_start, 0));
+    const size_t in_row = in_bytes / s.bh, out_row = out_bytes / s.bh;   // bytes per problem
+    const unsigned char *hQ = static_cast<const unsigned char *>(Q), *hK = static_cast<const unsigned char *>(K),
+                        *hV = static_cast<const unsigned char *>(V);
+    unsigned char *hO = static_cast<unsigned char *>(O);
+    for (int64_t ci = 0; ci < nchunk; ++ci) {
+        const int64_t p0 = s.bh * ci / nchunk, p1 = s.bh * (ci + 1) / nchunk;
+        const size_t off = in_row * p0, len = in_row * (p1 - p0);
+        HA_CUDA(h, cudaMemcpyAsync(dQ + off, hQ + off, len, cudaMemcpyHostToDevice, h->cs_in));
+        HA_CUDA(h, cudaMemcpyAsync(dK + off, hK + off, len, cudaMemcpyHostToDevice, h->cs_in));
+        HA_CUDA(h, cudaMemcpyAsync(dV + off, hV + off, len, cudaMemcpyHostToDevice, h->cs_in));
+        HA_CUDA(h, cudaEventRecord(h->pipe_ev[ci], h->cs_in));
+    }
+    for (int64_t ci = 0; ci < nchunk && rc == HA_OK; ++ci) {
+        const int64_t p0 = s.bh * ci / nchunk, p1 = s.bh * (ci + 1) / nchunk;
+        Shape sc = s;
+        sc.bh = p1 - p0;
+        HA_CUDA(h, cudaStreamWaitEvent(st, h->pipe_ev[ci], 0));
+        rc = run_forward(h, dQ + in_row * p0, dK + in_row * p0, dV + in_row * p0, dO + out_row * p0, sc, seed,
+                         h->opt.bh_offset + p0);
+        if (rc) break;
+        HA_CUDA(h, cudaEventRecord(h->pipe_ev[kChunks + ci], st));
+        HA_CUDA(h, cudaStreamWaitEvent(h->cs_out, h->pipe_ev[kChunks + ci], 0));
+        HA_CUDA(h, cudaMemcpyAsync(hO + out_row * p0, dO + out_row * p0, out_row * (p1 - p0),
+                                   cudaMemcpyDeviceToHost, h->cs_out));
+    }
     if (rc) {
         cudaStreamSynchronize(st);
+        cudaStreamSynchronize(h->cs_in);
+        cudaStreamSynchronize(h->cs_out);
         return rc;
     }
-    HA_CUDA(h, cudaMemcpyAsync(O, dO, out_bytes, cudaMemcpyDeviceToHost, st));
+    HA_CUDA(h, cudaStreamSynchronize(h->cs_out));
     HA_CUDA(h, cudaStreamSynchronize(st));
     return HA_OK;
 }
@@ -661,6 +707,11 @@ int hyper_attn_destroy(hyper_attn_t h) {
         if (h->pin) cudaFreeHost(h->pin);
         if (h->pin_free) cudaEventDestroy(h->pin_free);
         for (cudaEvent_t e : h->ev_pool) cudaEventDestroy(e);
+        if (h->cs_in) cudaStreamSynchronize(h->cs_in);
+        if (h->cs_out) cudaStreamSynchronize(h->cs_out);
+        for (cudaEvent_t e : h->pipe_ev) cudaEventDestroy(e);
+        if (h->cs_in) cudaStreamDestroy(h->cs_in);
+        if (h->cs_out) cudaStreamDestroy(h->cs_out);
     }
     delete h;
     return HA_OK;

@@ -165,6 +165,11 @@ struct Cfg {
     // product from queueing right behind the P.V that reads its buffer (a tensor-pipe stall; d = 128 is bound
     // by the pipe), one gives the second tile its next score tile sooner (d = 64 is bound by the softmax)
     static constexpr int kGroup = D == 64 ? 1 : 2;
+    // Two MMA issuers (score products on warp 1, P.V products on warp 2, the K loader also loading the Q
+    // tiles) instead of one issuer for both and a Q loader. Measured slower on this part for both head dims
+    // (a score product then waits for the completion of the P.V that last read its buffer, instead of queueing
+    // behind it), so it is off; the code is kept for other shapes and parts.
+    static constexpr bool kSplit = false;
     static constexpr int SEG = D == 64 ? 128 : 64;     // bytes per row segment of the staged output stores
     // d = 64: the epilogue stages its output rows in the item's own Q buffer (dead once the tile's last score
     // product has completed; the Q loader refills it only after the epilogue); d = 128 has a stage of its own
@@ -186,8 +191,8 @@ struct Cfg {
     static constexpr int bQFull = 0, bQEmpty = bQFull + 2 * QB, bKVFull = bQEmpty + 2 * QB,
                          bKVEmpty = bKVFull + NST, bWordFull = bKVEmpty + NST, bRowsFull = bWordFull + NST,
                          bSFull = bRowsFull + NST,
-                         bPFull = bSFull + R, bOReady = bPFull + R, bOFinal = bOReady + 4, bOFree = bOFinal + 2,
-                         bDrain = bOFree + 2, bQStage = bDrain + 1, kNumBars = bQStage + 2 * QB;
+                         bPFull = bSFull + R, bPVDone = bPFull + R, bPVDoneT = bPVDone + R, bOFree = bPVDoneT + 4,
+                         bDrain = bOFree + 2, bQStage = bDrain + 2, kNumBars = bQStage + 2 * QB;
     static constexpr int kTmemSlot = kBars + kNumBars * 8;
     static constexpr int kAbort = kTmemSlot + 4;
     static constexpr int kBytes = kAbort + 4;
@@ -298,12 +303,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
             mbar_init(bar(C::bSFull + b), 1);
             mbar_init(bar(C::bPFull + b), 128);
         }
-        for (int i = 0; i < 4; ++i) mbar_init(bar(C::bOReady + i), 1);
+        for (int b = 0; b < C::R; ++b) mbar_init(bar(C::bPVDone + b), 1);
+        for (int i = 0; i < 4; ++i) mbar_init(bar(C::bPVDoneT + i), 1);
         for (int t = 0; t < 2; ++t) {
-            mbar_init(bar(C::bOFinal + t), 1);
+            mbar_init(bar(C::bDrain + t), 1);
             mbar_init(bar(C::bOFree + t), 128);
         }
-        mbar_init(bar(C::bDrain), 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -333,50 +338,49 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
     constexpr int PPR = D / 8;             // 16-byte pieces per row
     constexpr int RPI = 32 / PPR;          // rows per warp instruction
 
-    if (warp == 2) {
-        // ------------------------------------------------------------------ Q loader
+    // Q tiles: tile t of an item into Q buffer qc mod QB of that tile, after the buffer's previous user (the
+    // tile's score products and, with the epilogue staged there, its epilogue) is done with it
+    int qc0 = 0, qc1 = 0;
+    auto load_q_tile = [&](const Item &x, int t) -> bool {
         const int rsub = lane / PPR, piece = lane % PPR, slab = piece >> 3, jp = piece & 7;
         int32_t *qperm = reinterpret_cast<int32_t *>(sm + C::kQPerm);
-        int qc0 = 0, qc1 = 0;
+        int &qc = t == 0 ? qc0 : qc1;
+        const int qb = qc % C::QB;
+        const int use = qc / C::QB;
+        if (use > 0 && !mbar_wait(bar(C::bQEmpty + t * C::QB + qb), (use - 1) & 1, abort_flag)) return false;
+        if (C::kStageInQ && use > 0 && !mbar_wait(bar(C::bQStage + t * C::QB + qb), (use - 1) & 1, abort_flag))
+            return false;
+        const uint32_t base = sbase + C::kQ + (t * C::QB + qb) * C::kTileBytes;
+        int64_t qbase;
+        const bool through_perm = a.mode == MODE_LEVEL;
+        if (through_perm) {
+            // the tile's 128 query rows: one 16-byte load per lane, staged in shared memory
+            const int32_t *pq = a.perm + (x.prob * 2) * a.lv.seg_len + x.blk * a.lv.bp + (x.pair * 2 + t) * 128;
+            __syncwarp();
+            reinterpret_cast<int4 *>(qperm)[lane] = reinterpret_cast<const int4 *>(pq)[lane];
+            __syncwarp();
+            qbase = x.bhi * a.n + x.node * a.lv.node_len + a.lv.q_off;
+        } else {
+            qbase = x.leaf_start + static_cast<int64_t>(t == 0 ? x.gt0 : x.gt1) * 128;
+        }
+#pragma unroll 8
+        for (int r0 = 0; r0 < 128; r0 += RPI) {
+            const int row = r0 + rsub;
+            const int64_t grow = qbase + (through_perm ? qperm[row] : row);
+            cp_async16(base + swz(slab, row, jp), a.Q + grow * D + piece * 8);
+        }
+        cp_async_arrive(bar(C::bQFull + t * C::QB + qb));
+        ++qc;
+        return true;
+    };
+
+    if (warp == 2 && !C::kSplit) {
+        // ------------------------------------------------------------------ Q loader
         bool ok = true;
         for (int64_t it = first; it < last && ok; it += stride) {
             const Item x = decode(a, it);
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {
-                if (!ok || !(t == 0 ? x.v0 : x.v1)) continue;
-                int &qc = t == 0 ? qc0 : qc1;
-                const int qb = qc % C::QB;
-                const int use = qc / C::QB;
-                if (use > 0 && !mbar_wait(bar(C::bQEmpty + t * C::QB + qb), (use - 1) & 1, abort_flag)) {
-                    ok = false;
-                    continue;
-                }
-                if (C::kStageInQ && use > 0 && !mbar_wait(bar(C::bQStage + t * C::QB + qb), (use - 1) & 1, abort_flag)) {
-                    ok = false;
-                    continue;
-                }
-                const uint32_t base = sbase + C::kQ + (t * C::QB + qb) * C::kTileBytes;
-                int64_t qbase;
-                const bool through_perm = a.mode == MODE_LEVEL;
-                if (through_perm) {
-                    // the tile's 128 query rows: one 16-byte load per lane, staged in shared memory
-                    const int32_t *pq = a.perm + (x.prob * 2) * a.lv.seg_len + x.blk * a.lv.bp + (x.pair * 2 + t) * 128;
-                    __syncwarp();
-                    reinterpret_cast<int4 *>(qperm)[lane] = reinterpret_cast<const int4 *>(pq)[lane];
-                    __syncwarp();
-                    qbase = x.bhi * a.n + x.node * a.lv.node_len + a.lv.q_off;
-                } else {
-                    qbase = x.leaf_start + static_cast<int64_t>(t == 0 ? x.gt0 : x.gt1) * 128;
-                }
-#pragma unroll 8
-                for (int r0 = 0; r0 < 128; r0 += RPI) {
-                    const int row = r0 + rsub;
-                    const int64_t grow = qbase + (through_perm ? qperm[row] : row);
-                    cp_async16(base + swz(slab, row, jp), a.Q + grow * D + piece * 8);
-                }
-                cp_async_arrive(bar(C::bQFull + t * C::QB + qb));
-                ++qc;
-            }
+            if (x.v0) ok = load_q_tile(x, 0);
+            if (ok && x.v1) ok = load_q_tile(x, 1);
         }
         cp_wait<0>();
         if (!ok) flag_status(a.status);
@@ -394,6 +398,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
         bool ok = true;
         for (int64_t it = first; it < last && ok; it += stride) {
             const Item x = decode(a, it);
+            if (C::kSplit) {   // this warp also loads the Q tiles (their buffers wait on items two back)
+                if (x.v0) ok = load_q_tile(x, 0);
+                if (ok && x.v1) ok = load_q_tile(x, 1);
+                if (!ok) break;
+            }
             // key rows of block blk and the compacted sample list of this item: the sampled columns whose key
             // lies outside block blk, in sample order (from the per-problem cache of samples and their blocks)
             int cnt = 0;
@@ -494,8 +503,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
         }
         cp_wait<0>();
         if (!ok) flag_status(a.status);
-    } else if (warp == 1) {
-        // ------------------------------------------------------------------ MMA issuer
+    } else if (warp == 1 && !C::kSplit) {
+        // ------------------------------------------------------------------ MMA issuer (score and P.V products)
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16(128, kKC, false, false);
             constexpr uint32_t idesc_pv = idesc_bf16(128, D, false, true);
@@ -513,7 +522,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                 int qb0, qb1;
                 int pre;
             };
-            int qc0 = 0, qc1 = 0, oc0 = 0, oc1 = 0;
+            int oc0 = 0, oc1 = 0;
+            uint32_t pvn0 = 0, pvn1 = 0;   // P.V products issued per tile
             bool ok = true;
             // wait for (blocking) or test (non-blocking) the Q tile of tile t of item f; false if not ready
             auto get_q = [&](Flight &f, int t, bool block) -> bool {
@@ -595,8 +605,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                     for (int kk = 0; kk < kKC / 16; ++kk)
                         mma_ts(od, tmem + buf * 128 + kk * 8, dv + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv,
                                (c > 0 || kk > 0) ? 1u : 0u);
-                    mma_commit(bar(C::bOReady + 2 * t + (c & 1)));
-                    if (c == (t == 0 ? x.nc0 : x.nc1) - 1) mma_commit(bar(C::bOFinal + t));
+                    // the tile's n-th P.V arrives on barrier 2t + (n & 1), phase n >> 1
+                    uint32_t &pvn = t == 0 ? pvn0 : pvn1;
+                    mma_commit(bar(C::bPVDoneT + 2 * t + (pvn & 1)));
+                    ++pvn;
                     // the chunk's stage is free once every tile that uses it has issued its P.V
                     const bool last_user = t == 1 || c >= x.nc1;
                     if (last_user) mma_commit(bar(C::bKVEmpty + slot));
@@ -633,6 +645,117 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
             mbar_wait(bar(C::bDrain), 0, &no_abort, 200000000ull);
         }
         __syncwarp();
+    } else if (warp == 1 && C::kSplit) {
+        // ------------------------------------------------------------------ score MMA issuer
+        // S of pair j (pair count of this CTA over all items) goes to ring buffer j mod R once P.V of pair j - R,
+        // the buffer's previous reader, has completed; runs ahead across items as far as the ring, the Q buffers
+        // and the K/V stages allow.
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = idesc_bf16(128, kKC, false, false);
+            // descriptors are built once; an MMA only adds a byte offset >> 4 to the start-address field
+            const uint64_t dq0 = smem_desc(sbase + C::kQ, 16, 1024);
+            const uint64_t dk0 = smem_desc(sbase + C::kK, 16, 1024);
+            uint32_t j = 0, g = 0, kv_ready = 0;
+            int sq0 = 0, sq1 = 0;   // Q tiles taken per tile
+            bool ok = true;
+            for (int64_t it = first; it < last && ok; it += stride) {
+                const Item x = decode(a, it);
+                int qb0 = -1, qb1 = -1;
+                for (int k = 0; k < x.npairs; ++k, ++j) {
+                    int t, c;
+                    pair_tc(x, k, t, c);
+                    int &qb = t == 0 ? qb0 : qb1;
+                    if (qb < 0) {
+                        int &qc = t == 0 ? sq0 : sq1;
+                        if (!mbar_wait(bar(C::bQFull + t * C::QB + qc % C::QB), (qc / C::QB) & 1, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        qb = qc % C::QB;
+                        ++qc;
+                    }
+                    const uint32_t gc = g + static_cast<uint32_t>(c);
+                    const int slot = static_cast<int>(gc % C::NST);
+                    if (gc >= kv_ready) {   // chunks arrive in order: wait once per chunk
+                        if (!mbar_wait(bar(C::bKVFull + slot), (gc / C::NST) & 1, abort_flag)) { ok = false; break; }
+                        kv_ready = gc + 1;
+                    }
+                    const int buf = static_cast<int>(j % C::R);
+                    if (j >= static_cast<uint32_t>(C::R) &&
+                        !mbar_wait(bar(C::bPVDone + buf), (j / C::R - 1) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t dq = dq0 + static_cast<uint64_t>(((t * C::QB + qb) * C::kTileBytes) >> 4);
+                    const uint64_t dk = dk0 + static_cast<uint64_t>((slot * C::kTileBytes) >> 4);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint64_t off = static_cast<uint64_t>(((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4);
+                        mma_ss(tmem + buf * 128, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(bar(C::bSFull + buf));
+                    // last score tile of this query tile in this item: its Q buffer may be refilled
+                    if (c == (t == 0 ? x.nc0 : x.nc1) - 1) mma_commit(bar(C::bQEmpty + t * C::QB + qb));
+                }
+                g += static_cast<uint32_t>(x.nc_max);
+            }
+            if (!ok) flag_status(a.status);
+            mma_commit(bar(C::bDrain));   // this thread's MMAs complete before TMEM is released
+            volatile int no_abort = 0;
+            mbar_wait(bar(C::bDrain), 0, &no_abort, 200000000ull);
+        }
+        __syncwarp();
+    } else if (warp == 2 && C::kSplit) {
+        // ------------------------------------------------------------------ P.V MMA issuer
+        // O_t += P(j) V(chunk) once the softmax has written P of pair j; then signals the tile's P.V count
+        // (softmax: rescale and epilogue), the ring buffer (score issuer) and, after the chunk's last user, the
+        // K/V stage.
+        if (lane == 0) {
+            constexpr uint32_t idesc_pv = idesc_bf16(128, D, false, true);
+            const uint64_t dv0 = smem_desc(sbase + C::kV, 128 * 128, 1024);
+            uint32_t j = 0, g = 0;
+            uint32_t pvn0 = 0, pvn1 = 0;   // P.V products issued per tile
+            int oc0 = 0, oc1 = 0;
+            bool ok = true;
+            for (int64_t it = first; it < last && ok; it += stride) {
+                const Item x = decode(a, it);
+                for (int k = 0; k < x.npairs; ++k, ++j) {
+                    int t, c;
+                    pair_tc(x, k, t, c);
+                    const int buf = static_cast<int>(j % C::R);
+                    if (!mbar_wait(bar(C::bPFull + buf), (j / C::R) & 1, abort_flag)) { ok = false; break; }
+                    const int oc = t == 0 ? oc0 : oc1;
+                    if (c == 0 && oc > 0 && !mbar_wait(bar(C::bOFree + t), (oc - 1) & 1, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t gc = g + static_cast<uint32_t>(c);
+                    const int slot = static_cast<int>(gc % C::NST);
+                    // V of chunk c arrived with K (one barrier per stage), which S of this pair waited for
+                    const uint64_t dv = dv0 + static_cast<uint64_t>((slot * C::kTileBytes) >> 4);
+                    const uint32_t od = tmem + C::kOCol + t * D;
+#pragma unroll
+                    for (int kk = 0; kk < kKC / 16; ++kk)
+                        mma_ts(od, tmem + buf * 128 + kk * 8, dv + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv,
+                               (c > 0 || kk > 0) ? 1u : 0u);
+                    // the tile's barrier first, then the ring buffer's: a waiter that has seen the buffer free may
+                    // rely on the tile's barrier having arrived
+                    uint32_t &pvn = t == 0 ? pvn0 : pvn1;
+                    mma_commit(bar(C::bPVDoneT + 2 * t + (pvn & 1)));
+                    ++pvn;
+                    mma_commit(bar(C::bPVDone + buf));
+                    // the chunk's stage is free once every tile that uses it has issued its P.V
+                    if (t == 1 || c >= x.nc1) mma_commit(bar(C::bKVEmpty + slot));
+                }
+                if (x.v0) ++oc0;
+                if (x.v1) ++oc1;
+                g += static_cast<uint32_t>(x.nc_max);
+            }
+            if (!ok) flag_status(a.status);
+            mma_commit(bar(C::bDrain + 1));
+            volatile int no_abort = 0;
+            mbar_wait(bar(C::bDrain + 1), 0, &no_abort, 200000000ull);
+        }
+        __syncwarp();
     } else if (warp >= 4) {
         // ------------------------------------------------------------------ softmax + epilogue
         const int t = (warp - 4) >> 2;
@@ -641,7 +764,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
         const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
         const uint32_t tO = trow + C::kOCol + t * D;
         uint32_t kp = 0, g = 0;
-        int hp0 = 0, hp1 = 0, fin = 0;               // P handoffs per chunk parity; epilogues done
+        uint32_t pvt = 0;                            // P.V products of this tile before the current item
         int qn = 0;                                  // items of this tile so far (its Q buffer is qn mod QB)
         bool ok = true;
         for (int64_t it = first; it < last && ok; it += stride) {
@@ -707,9 +830,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                 l *= alpha;
                 if (c > 0 && __any_sync(0xffffffffu, grow)) {
                     // O holds P.V of chunks 0..c-1: wait for the last of them (chunk c-1) before scaling it
-                    const int pp = (c - 1) & 1;
-                    const int use = (pp ? hp1 : hp0) - 1;
-                    if (!mbar_wait(bar(C::bOReady + 2 * t + pp), use & 1, abort_flag)) ok = false;
+                    const uint32_t nprev = pvt + static_cast<uint32_t>(c) - 1;
+                    if (!mbar_wait(bar(C::bPVDoneT + 2 * t + (nprev & 1)), (nprev >> 1) & 1, abort_flag)) ok = false;
                     if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
                     tc_fence_after();
 #pragma unroll
@@ -759,13 +881,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                 tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(bar(C::bPFull + buf));
-                if (c & 1) ++hp1; else ++hp0;
             }
             if (!ok) break;
             // epilogue: wait for the tile's last P.V of this item, then write the row
-            if (!mbar_wait(bar(C::bOFinal + t), fin & 1, abort_flag)) ok = false;
+            const uint32_t nlast = pvt + static_cast<uint32_t>(my_nc) - 1;
+            if (!mbar_wait(bar(C::bPVDoneT + 2 * t + (nlast & 1)), (nlast >> 1) & 1, abort_flag)) ok = false;
             if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
-            ++fin;
+            pvt += static_cast<uint32_t>(my_nc);
             tc_fence_after();
             const float inv_l = 1.0f / l;
             const float Lrow = (m_run + __log2f(l)) * kLn2;   // natural log of the row's normaliser

@@ -334,11 +334,17 @@ def run_ours(args, w: wl.Workload):
     avg_ms = dom_ms / (args.steps * groups)
     byts, flops = algorithmic(w, dom)
     if flops > 0 and dom in ("attn", "causal_base"):
-        if family == "tc":
-            bound, peak, unit = "tensor", peaks["bf16_tflops"], "TFLOP/s"
+        # the binding roof is the one with the larger ideal time: algorithmic bytes at HBM peak or FLOPs at the
+        # compute peak (tensor for the tcgen05 kernels, FP32 ALU for the SIMT ones)
+        cpeak = peaks["bf16_tflops"] if family == "tc" else FP32_SIMT_PEAK_TFLOPS
+        t_compute = flops / (cpeak * 1e12)
+        t_memory = byts / (peaks["hbm_gbs"] * 1e9)
+        if t_compute >= t_memory:
+            bound, peak, unit = ("tensor" if family == "tc" else "alu"), cpeak, "TFLOP/s"
+            achieved = flops / (avg_ms * 1e-3) / 1e12
         else:
-            bound, peak, unit = "alu", FP32_SIMT_PEAK_TFLOPS, "TFLOP/s"
-        achieved = flops / (avg_ms * 1e-3) / 1e12
+            bound, peak, unit = "hbm", peaks["hbm_gbs"], "GB/s"
+            achieved = byts / (avg_ms * 1e-3) / 1e9
     else:
         bound, peak, unit = "hbm", peaks["hbm_gbs"], "GB/s"
         achieved = byts / (avg_ms * 1e-3) / 1e9

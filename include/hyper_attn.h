@@ -102,8 +102,12 @@ HA_API int hyper_attn_forward(hyper_attn_t h, const void *Q, const void *K, cons
 
 /*
  * Same computation with HOST buffers: copies Q, K, V to handle-owned device buffers, runs the forward
- * pass, copies O back and waits for the stream. Returns when O is valid on the host. Page-locked host
- * memory is copied asynchronously; pageable memory is staged by the CUDA runtime.
+ * pass, copies O back and waits. Returns when O is valid on the host. The (batch, head) problems go
+ * through in up to 8 contiguous groups so that host-to-device copies, the forward pass (on the handle's
+ * stream, after any work already queued there) and device-to-host copies of different groups overlap, on
+ * two copy streams the handle owns; the result equals one pass over all problems (each group's draws are
+ * keyed by global problem index). The overlap needs page-locked host memory; pageable memory is staged by
+ * the CUDA runtime and mostly serialises. With debug captures on, all problems form one group.
  */
 HA_API int hyper_attn_forward_host(hyper_attn_t h, const void *Q, const void *K, const void *V, void *O,
                             int64_t n, int d, int heads, int block, int m, int r, int causal, uint64_t seed);

@@ -149,13 +149,23 @@ def test_bf16_output(ha):
         assert rel_err(got[h], ref) < 2e-3 + 2.0 ** -9
 
 
-def test_forward_host_matches_device(ha):
-    n, d, bh, block, m, r, seed = 2048, 64, 2, 128, 64, 6, 77
+@pytest.mark.parametrize("n,d,bh,block,m,r,causal,base", [
+    (2048, 64, 2, 128, 64, 6, False, 0),
+    (1024, 128, 11, 256, 128, 7, False, 0),     # 11 problems in 8 uneven groups
+    (2048, 64, 5, 128, 64, 6, True, 512),
+])
+def test_forward_host_matches_device(ha, n, d, bh, block, m, r, causal, base):
+    """The host-buffer entry point (problem groups pipelined over copy streams) equals the device one."""
+    seed = 77
     Qh, Kh, Vh = wl.make_inputs(n, d, bh, data_seed=seed, dtype="bf16")
-    dev = run_gpu(ha, Qh, Kh, Vh, n=n, d=d, bh=bh, block=block, m=m, r=r, causal=False, seed=seed, out_dtype="bf16",
-                  debug=False)
+    dev = run_gpu(ha, Qh, Kh, Vh, n=n, d=d, bh=bh, block=block, m=m, r=r, causal=causal, seed=seed, base=base,
+                  out_dtype="bf16", debug=False)
     Oh = np.zeros((bh, n, d), np.uint16)
-    ha.forward_host(Qh, Kh, Vh, Oh, n=n, d=d, heads=bh, block=block, m=m, r=r, causal=False, seed=seed)
+    Qp, Kp, Vp, Op = (torch.from_numpy(x.view(np.int16)).pin_memory() for x in (Qh, Kh, Vh, Oh))
+    ha.forward_host(Qp, Kp, Vp, Op, n=n, d=d, heads=bh, block=block, m=m, r=r, causal=causal, seed=seed)
+    assert np.array_equal(wl.as_f32(Op.numpy().view(np.uint16)).astype(np.float64), dev)
+    # pageable buffers take the same path
+    ha.forward_host(Qh, Kh, Vh, Oh, n=n, d=d, heads=bh, block=block, m=m, r=r, causal=causal, seed=seed)
     assert np.array_equal(wl.as_f32(Oh).astype(np.float64), dev)
 
 

@@ -36,15 +36,15 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # taken from is unchanged (sha256 of the file at capture time).
 TRAFFIC = {
     # 4-head capture of the 32-head workload (the full one is too large for a multi-pass capture), scaled x8
-    # by the rows processed: attention 205.8 MB read + 42.6 MB written per 4-head launch; hash 134.2 + 5.0 MB.
+    # by the rows processed: attention 205.8 MB read + 43.2 MB written per 4-head launch; hash 134.2 + 6.2 MB.
     ("attn", "long_bf16_n131072", "tc"): {
         "file": "ha_attn_tc.cu",
-        "sha256": "9c1760df52f2b25c6a9df7686f44075be3f5e664465c7ffaaf72aeacfd2ed29b",
-        "bytes": 8 * (205_848_064 + 42_623_488)},
+        "sha256": "acec50e69c597030cd598123d0351faa91bcca66d20f08407371f516b6b506aa",
+        "bytes": 8 * (205_809_408 + 43_212_288)},
     ("hash", "long_bf16_n131072", "tc"): {
         "file": "ha_hash.cu",
-        "sha256": "b86668b0d82f1c4fc5e060be3a59b195a331f6726fa6ed7fde3726287ce783fb",
-        "bytes": 8 * (134_234_624 + 4_986_112)},
+        "sha256": "4590cdf32028d354a14840822c657310cf7c55c4363a9d576b207e5aa9b08c08",
+        "bytes": 8 * (134_242_560 + 6_169_856)},
 }
 
 

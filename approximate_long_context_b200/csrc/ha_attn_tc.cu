@@ -158,7 +158,11 @@ __device__ __forceinline__ void pair_tc(const Item &x, int k, int &t, int &c) {
 
 template <int D>
 struct Cfg {
-    static constexpr int R = D == 64 ? 3 : 2;          // S ring buffers
+    // d = 64: P in TMEM buffers of its own (one per tile), so that the score tile of pair k + R may overwrite
+    // S of pair k as soon as the softmax has read it, before P of pair k exists (TMEM: 2 x 128 S columns,
+    // 2 x 64 P columns, 2 x 64 O columns). d = 128 writes P over its S (TMEM: 2 x 128 S, 2 x 128 O).
+    static constexpr bool kSepP = D == 64;
+    static constexpr int R = 2;                        // S ring buffers
     static constexpr int QB = D == 64 ? 2 : 1;         // Q buffers per tile
     static constexpr int NST = D == 64 ? 4 : 2;        // K/V stages
     // P.V products issued per group before the score products that reuse their buffers: two keep a score
@@ -174,7 +178,8 @@ struct Cfg {
     // d = 64: the epilogue stages its output rows in the item's own Q buffer (dead once the tile's last score
     // product has completed; the Q loader refills it only after the epilogue); d = 128 has a stage of its own
     static constexpr bool kStageInQ = D == 64;
-    static constexpr int kOCol = R * 128;              // first O column
+    static constexpr int kPCol = R * 128;              // P of tile t at [kPCol + 64 t, kPCol + 64 (t + 1)) (kSepP)
+    static constexpr int kOCol = R * 128 + (kSepP ? 128 : 0);   // first O column
     static constexpr int kTileBytes = 128 * D * 2;     // 128 rows of bf16 (a Q tile, a K or a V chunk)
     static constexpr int kQ = 0;
     static constexpr int kK = kQ + 2 * QB * kTileBytes;
@@ -192,7 +197,8 @@ struct Cfg {
                          bKVEmpty = bKVFull + NST, bWordFull = bKVEmpty + NST, bRowsFull = bWordFull + NST,
                          bSFull = bRowsFull + NST,
                          bPFull = bSFull + R, bPVDone = bPFull + R, bPVDoneT = bPVDone + R, bOFree = bPVDoneT + 4,
-                         bDrain = bOFree + 2, bQStage = bDrain + 2, kNumBars = bQStage + 2 * QB;
+                         bDrain = bOFree + 2, bQStage = bDrain + 2, bSFree = bQStage + 2 * QB, bPFullT = bSFree + R,
+                         kNumBars = bPFullT + 2;
     static constexpr int kTmemSlot = kBars + kNumBars * 8;
     static constexpr int kAbort = kTmemSlot + 4;
     static constexpr int kBytes = kAbort + 4;
@@ -302,9 +308,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
         for (int b = 0; b < C::R; ++b) {
             mbar_init(bar(C::bSFull + b), 1);
             mbar_init(bar(C::bPFull + b), 128);
+            mbar_init(bar(C::bSFree + b), 128);    // kSepP: the softmax threads of the pair's tile have read S
         }
         for (int b = 0; b < C::R; ++b) mbar_init(bar(C::bPVDone + b), 1);
         for (int i = 0; i < 4; ++i) mbar_init(bar(C::bPVDoneT + i), 1);
+        for (int t = 0; t < 2; ++t) mbar_init(bar(C::bPFullT + t), 128);   // kSepP: P of a tile's pair written
         for (int t = 0; t < 2; ++t) {
             mbar_init(bar(C::bDrain + t), 1);
             mbar_init(bar(C::bOFree + t), 128);
@@ -587,6 +595,24 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                     nxt.qb0 = -1; nxt.qb1 = -1; nxt.pre = 0;
                 }
                 bool look = have_next;   // look-ahead into the next item still possible
+                // the score tile R pairs ahead, in this item or (look-ahead) in the next one
+                auto issue_ahead = [&](int ka) {
+                    if (ka < np) {
+                        ok = issue_s(cur, ka);
+                    } else if (look) {
+                        const int kn = ka - np;
+                        if (kn == nxt.pre && kn < nxt.x.npairs) {
+                            int tn, cn;
+                            pair_tc(nxt.x, kn, tn, cn);
+                            // with one Q buffer per tile, the next Q is loaded only after this item's last S:
+                            // take it only if it is already there
+                            if (get_q(nxt, tn, C::QB > 1)) ok = issue_s(nxt, kn);
+                            else look = false;
+                        } else {
+                            look = false;
+                        }
+                    }
+                };
                 for (int k = 0; k < np && ok; ++k) {
                     int t, c;
                     pair_tc(x, k, t, c);
@@ -594,7 +620,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                     const int slot = static_cast<int>(gc % C::NST);
                     const uint32_t kk_all = cur.kp + static_cast<uint32_t>(k);
                     const int buf = static_cast<int>(kk_all % C::R);
-                    if (!mbar_wait(bar(C::bPFull + buf), (kk_all / C::R) & 1, abort_flag)) { ok = false; break; }
+                    uint32_t &pvn = t == 0 ? pvn0 : pvn1;
+                    if (C::kSepP) {
+                        // S of pair k has been read: its buffer takes the score tile R pairs ahead
+                        if (!mbar_wait(bar(C::bSFree + buf), (kk_all / C::R) & 1, abort_flag)) { ok = false; break; }
+                        issue_ahead(k + C::R);
+                        if (!ok) break;
+                        if (!mbar_wait(bar(C::bPFullT + t), pvn & 1, abort_flag)) { ok = false; break; }
+                    } else if (!mbar_wait(bar(C::bPFull + buf), (kk_all / C::R) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
                     const int oc = t == 0 ? oc0 : oc1;
                     if (c == 0 && oc > 0 && !mbar_wait(bar(C::bOFree + t), (oc - 1) & 1, abort_flag)) { ok = false; break; }
                     tc_fence_after();
@@ -602,37 +638,21 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                     const uint64_t dv = dv0 + static_cast<uint64_t>((slot * C::kTileBytes) >> 4);
                     const uint32_t od = tmem + C::kOCol + t * D;
 #pragma unroll
-                    for (int kk = 0; kk < kKC / 16; ++kk)
-                        mma_ts(od, tmem + buf * 128 + kk * 8, dv + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv,
-                               (c > 0 || kk > 0) ? 1u : 0u);
-                    // the tile's n-th P.V arrives on barrier 2t + (n & 1), phase n >> 1
-                    uint32_t &pvn = t == 0 ? pvn0 : pvn1;
+                    for (int kk = 0; kk < kKC / 16; ++kk) {
+                        const uint32_t pa = C::kSepP ? tmem + C::kPCol + t * 64 + kk * 8 : tmem + buf * 128 + kk * 8;
+                        mma_ts(od, pa, dv + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv, (c > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    // the tile's n-th P.V arrives on barrier 2t + (n & 1), phase n >> 1 (with P apart, this also
+                    // frees the tile's P buffer)
                     mma_commit(bar(C::bPVDoneT + 2 * t + (pvn & 1)));
                     ++pvn;
                     // the chunk's stage is free once every tile that uses it has issued its P.V
                     const bool last_user = t == 1 || c >= x.nc1;
                     if (last_user) mma_commit(bar(C::bKVEmpty + slot));
-                    // the ring buffers of this pair group (kGroup = 2: pairs k-1 and k, or k alone at an odd end) are
-                    // free again: fill them with the score tiles R pairs ahead
-                    if (C::kGroup == 1 || (k & 1) || k == np - 1) {
-                        for (int kg = (C::kGroup == 2 && (k & 1)) ? k - 1 : k; kg <= k && ok; ++kg) {
-                            const int ka = kg + C::R;
-                            if (ka < np) {
-                                ok = issue_s(cur, ka);
-                            } else if (look) {
-                                const int kn = ka - np;
-                                if (kn == nxt.pre && kn < nxt.x.npairs) {
-                                    int tn, cn;
-                                    pair_tc(nxt.x, kn, tn, cn);
-                                    // with one Q buffer per tile, the next Q is loaded only after this item's last S:
-                                    // take it only if it is already there
-                                    if (get_q(nxt, tn, C::QB > 1)) ok = issue_s(nxt, kn);
-                                    else look = false;
-                                } else {
-                                    look = false;
-                                }
-                            }
-                        }
+                    // P over S: the ring buffers of this pair group (kGroup = 2: pairs k-1 and k, or k alone at an
+                    // odd end) are free again: fill them with the score tiles R pairs ahead
+                    if (!C::kSepP && (C::kGroup == 1 || (k & 1) || k == np - 1)) {
+                        for (int kg = (C::kGroup == 2 && (k & 1)) ? k - 1 : k; kg <= k && ok; ++kg) issue_ahead(kg + C::R);
                     }
                 }
                 if (x.v0) ++oc0;
@@ -848,14 +868,27 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                 m_run = m_new;
                 const float off = w2 - m_run;
                 float l0 = 0.0f, l1 = 0.0f;
-                // pass 2: P = 2^(x - m_run) in bf16 over the first 64 columns of the buffer (keys 0-63 land in
-                // columns 0-31, already read; keys 64-127 in columns 32-63, read by the first half)
+                // pass 2: P = 2^(x - m_run) in bf16, 64 columns: over the first 64 columns of the S buffer (keys
+                // 0-63 land in columns 0-31, already read; keys 64-127 in columns 32-63, read by the first half),
+                // or (kSepP) into the tile's P buffer once the tile's previous P.V has read it
+                const uint32_t tP = C::kSepP ? trow + C::kPCol + t * 64 : tS;
+                if (C::kSepP && pvt + static_cast<uint32_t>(c) > 0) {
+                    const uint32_t nprev = pvt + static_cast<uint32_t>(c) - 1;
+                    if (!mbar_wait(bar(C::bPVDoneT + 2 * t + (nprev & 1)), (nprev >> 1) & 1, abort_flag)) ok = false;
+                    if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
+                    tc_fence_after();
+                }
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     uint32_t va[32], vb[32];
                     tmem_ld32(tS + h * 64, va);
                     tmem_ld32(tS + h * 64 + 32, vb);
                     tmem_ld_wait();
+                    if (C::kSepP && h == 1) {
+                        // all of S has been read: the buffer may take the next score tile
+                        tc_fence_before();
+                        mbar_arrive(bar(C::bSFree + buf));
+                    }
                     if (masked) {
 #pragma unroll
                         for (int e = 0; e < 32; ++e) {
@@ -875,12 +908,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                         pk[e] = pack_bf16x2(p0, p1);
                         pk[16 + e] = pack_bf16x2(p2, p3);
                     }
-                    tmem_st32(tS + h * 32, pk);
+                    tmem_st32(tP + h * 32, pk);
                 }
                 l += l0 + l1;
                 tmem_st_wait();
                 tc_fence_before();
-                mbar_arrive(bar(C::bPFull + buf));
+                mbar_arrive(bar(C::kSepP ? C::bPFullT + t : C::bPFull + buf));
             }
             if (!ok) break;
             // epilogue: wait for the tile's last P.V of this item, then write the row

@@ -99,10 +99,11 @@ struct Item {
 
 // Item index -> item. Item counts, problem counts and their factors are below 2^31 (checked on the host), so the
 // divisions are 32-bit.
+template <int MODE>
 __device__ __forceinline__ Item decode(const TcArgs &a, int64_t it64) {
     Item x{};
     const uint32_t it = static_cast<uint32_t>(it64);
-    if (a.mode == MODE_LEVEL) {
+    if (MODE == MODE_LEVEL) {
         const uint32_t prob = it / a.per_outer;
         const uint32_t rem = it - prob * a.per_outer;
         const uint32_t ppb = static_cast<uint32_t>(a.pairs_per_block);
@@ -279,7 +280,10 @@ __device__ __forceinline__ uint32_t swz(int slab, int row, int j) {
     return static_cast<uint32_t>(slab * (128 * 128) + row * 128 + ((j ^ (row & 7)) << 4));
 }
 
-template <int D>
+// MODE (MODE_LEVEL or MODE_CAUSAL) is a compile-time parameter: each instance holds only its own mode's loads,
+// masks and epilogue, which keeps the instruction footprint of the concurrently running roles small (measured:
+// about 4% faster than one instance for both modes).
+template <int D, int MODE>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
     using C = Cfg<D>;
     extern __shared__ unsigned char smem_raw[];
@@ -332,7 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
     // LEVEL items all cost the same: each CTA takes a contiguous range, so consecutive items share a problem
     // and its cached samples. CAUSAL items are ordered heaviest first and dealt round-robin.
     int64_t first, last, stride;
-    if (a.mode == MODE_LEVEL) {
+    if (MODE == MODE_LEVEL) {
         const int64_t per = (a.items + gridDim.x - 1) / gridDim.x;
         first = static_cast<int64_t>(blockIdx.x) * per;
         last = min(a.items, first + per);
@@ -360,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
             return false;
         const uint32_t base = sbase + C::kQ + (t * C::QB + qb) * C::kTileBytes;
         int64_t qbase;
-        const bool through_perm = a.mode == MODE_LEVEL;
+        const bool through_perm = MODE == MODE_LEVEL;
         if (through_perm) {
             // the tile's 128 query rows: one 16-byte load per lane, staged in shared memory
             const int32_t *pq = a.perm + (x.prob * 2) * a.lv.seg_len + x.blk * a.lv.bp + (x.pair * 2 + t) * 128;
@@ -386,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
         // ------------------------------------------------------------------ Q loader
         bool ok = true;
         for (int64_t it = first; it < last && ok; it += stride) {
-            const Item x = decode(a, it);
+            const Item x = decode<MODE>(a, it);
             if (x.v0) ok = load_q_tile(x, 0);
             if (ok && x.v1) ok = load_q_tile(x, 1);
         }
@@ -405,7 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
         uint32_t g = 0;
         bool ok = true;
         for (int64_t it = first; it < last && ok; it += stride) {
-            const Item x = decode(a, it);
+            const Item x = decode<MODE>(a, it);
             if (C::kSplit) {   // this warp also loads the Q tiles (their buffers wait on items two back)
                 if (x.v0) ok = load_q_tile(x, 0);
                 if (ok && x.v1) ok = load_q_tile(x, 1);
@@ -415,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
             // lies outside block blk, in sample order (from the per-problem cache of samples and their blocks)
             int cnt = 0;
             int64_t kbase = 0;
-            if (a.mode == MODE_LEVEL) {
+            if (MODE == MODE_LEVEL) {
                 kbase = x.bhi * a.n + x.node * a.lv.node_len;
                 const int32_t *pkg = a.perm + (x.prob * 2 + 1) * a.lv.seg_len + x.blk * a.lv.bp;
                 __syncwarp();
@@ -449,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                 int valid_cols = kKC;
                 int kind;   // 0: block chunk (through the key permutation), 1: sample chunk, 2: contiguous
                 int u0 = 0;
-                if (a.mode == MODE_LEVEL) {
+                if (MODE == MODE_LEVEL) {
                     if (c < a.nb) {
                         kind = 0;
                     } else {
@@ -465,7 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                     mbar_arrive(bar(C::bWordFull + slot));
                 }
                 // the chunk's 128 global rows, published for the V loader
-                const int64_t cbase = a.mode == MODE_LEVEL ? kbase : x.leaf_start + static_cast<int64_t>(c) * kKC;
+                const int64_t cbase = (MODE == MODE_LEVEL) ? kbase : x.leaf_start + static_cast<int64_t>(c) * kKC;
                 int32_t *rows = stage_rows + slot * 128;
                 for (int row = lane; row < kKC; row += 32) {
                     int32_t loc;
@@ -495,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
         uint32_t g = 0;
         bool ok = true;
         for (int64_t it = first; it < last && ok; it += stride) {
-            const Item x = decode(a, it);
+            const Item x = decode<MODE>(a, it);
             for (int c = 0; c < x.nc_max; ++c, ++g) {
                 const int slot = static_cast<int>(g % C::NST);
                 if (!mbar_wait(bar(C::bRowsFull + slot), (g / C::NST) & 1, abort_flag)) { ok = false; break; }
@@ -574,7 +578,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
             Flight cur{}, nxt{};
             bool have_next = false;
             if (first < last) {
-                cur.x = decode(a, first);
+                cur.x = decode<MODE>(a, first);
                 cur.g = 0; cur.kp = 0; cur.qb0 = -1; cur.qb1 = -1; cur.pre = 0;
             }
             for (int64_t it = first; it < last && ok; it += stride) {
@@ -589,7 +593,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                 }
                 have_next = it + stride < last;
                 if (have_next) {
-                    nxt.x = decode(a, it + stride);
+                    nxt.x = decode<MODE>(a, it + stride);
                     nxt.g = cur.g + x.nc_max;
                     nxt.kp = cur.kp + np;
                     nxt.qb0 = -1; nxt.qb1 = -1; nxt.pre = 0;
@@ -679,7 +683,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
             int sq0 = 0, sq1 = 0;   // Q tiles taken per tile
             bool ok = true;
             for (int64_t it = first; it < last && ok; it += stride) {
-                const Item x = decode(a, it);
+                const Item x = decode<MODE>(a, it);
                 int qb0 = -1, qb1 = -1;
                 for (int k = 0; k < x.npairs; ++k, ++j) {
                     int t, c;
@@ -739,7 +743,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
             int oc0 = 0, oc1 = 0;
             bool ok = true;
             for (int64_t it = first; it < last && ok; it += stride) {
-                const Item x = decode(a, it);
+                const Item x = decode<MODE>(a, it);
                 for (int k = 0; k < x.npairs; ++k, ++j) {
                     int t, c;
                     pair_tc(x, k, t, c);
@@ -788,13 +792,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
         int qn = 0;                                  // items of this tile so far (its Q buffer is qn mod QB)
         bool ok = true;
         for (int64_t it = first; it < last && ok; it += stride) {
-            const Item x = decode(a, it);
+            const Item x = decode<MODE>(a, it);
             const bool my_valid = t == 0 ? x.v0 : x.v1;
             const int my_nc = t == 0 ? x.nc0 : x.nc1;
             const int my_gt = t == 0 ? x.gt0 : x.gt1;
             if (!my_valid) { kp += x.npairs; g += x.nc_max; continue; }
             int64_t qloc = 0;
-            if (a.mode == MODE_LEVEL) {
+            if (MODE == MODE_LEVEL) {
                 const int64_t pos = x.blk * a.lv.bp + (x.pair * 2 + t) * 128 + r;
                 qloc = a.perm[(x.prob * 2) * a.lv.seg_len + pos];   // consumed by the epilogue
             }
@@ -807,7 +811,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                 // column bound: columns > bound are masked (bound >= 127: none)
                 int bound = kKC - 1;
                 float w2 = 0.0f;
-                if (a.mode == MODE_LEVEL) {
+                if (MODE == MODE_LEVEL) {
                     if (c >= a.nb) {
                         const uint32_t gc = g + c;
                         const int slot = static_cast<int>(gc % C::NST);
@@ -936,7 +940,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                     for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(o[e]) * scale;
                 };
             };
-            if (a.mode == MODE_LEVEL) {
+            if (MODE == MODE_LEVEL) {
                 const int64_t N = a.lv.seg_len;
                 if (a.lv.level == 0) {
                     const int64_t orow = x.bhi * a.n + a.lv.q_off + x.node * a.lv.node_len + qloc;
@@ -1032,13 +1036,13 @@ int num_sms() {
     return sms;
 }
 
-template <int D>
+template <int D, int MODE>
 int launch_tc(const void *Q, const void *K, const void *V, TcArgs args, cudaStream_t st) {
     args.Q = static_cast<const uint16_t *>(Q);
     args.K = static_cast<const uint16_t *>(K);
     args.V = static_cast<const uint16_t *>(V);
     const size_t smem = Cfg<D>::kBytes + 1024;
-    auto kern = attn_tc_kernel<D>;
+    auto kern = attn_tc_kernel<D, MODE>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
         return -1;
     const int64_t grid = args.items < num_sms() ? args.items : num_sms();
@@ -1048,8 +1052,10 @@ int launch_tc(const void *Q, const void *K, const void *V, TcArgs args, cudaStre
 }
 
 int dispatch(int d, const void *Q, const void *K, const void *V, const TcArgs &args, cudaStream_t st) {
-    if (d == 64) return launch_tc<64>(Q, K, V, args, st);
-    if (d == 128) return launch_tc<128>(Q, K, V, args, st);
+    const bool level = args.mode == MODE_LEVEL;
+    if (d == 64) return level ? launch_tc<64, MODE_LEVEL>(Q, K, V, args, st) : launch_tc<64, MODE_CAUSAL>(Q, K, V, args, st);
+    if (d == 128)
+        return level ? launch_tc<128, MODE_LEVEL>(Q, K, V, args, st) : launch_tc<128, MODE_CAUSAL>(Q, K, V, args, st);
     return -2;
 }
 

@@ -19,11 +19,13 @@
 //  g sees key chunks 0..g, the last one with the inclusive causal mask. Items run heaviest first.
 //
 // Work unit of the MMA and softmax roles: a "pair" (query tile t, key chunk c) of 128 x 128 scores. The
-// pairs of an item run c-major, t-minor. S of pair k lives in TMEM buffer k mod R of a ring of R buffers of
-// 128 columns; the softmax overwrites it with P (bf16, its first 64 columns) and the P.V product reads P
-// from TMEM. The MMA issues S of pair k+R right after P.V of pair k (same buffer, issued in order), so up
-// to R score tiles are in flight while the softmax works. (On this part an M=128, K=16 MMA costs about
-// the same for N = 64 and N = 128, so 128-key chunks halve the cost of the score products.)
+// pairs of an item run c-major, t-minor; j counts pairs over a CTA's items. S of pair j lives in TMEM buffer
+// j mod R of a ring of R = 2 buffers of 128 columns. d = 64: the softmax writes P (bf16) to a TMEM buffer of
+// its tile, and S of pair j + 2 is issued as soon as the softmax has read S of pair j. d = 128: P overwrites
+// the first 64 columns of its S buffer, and S of pair j + 2 is issued right after the P.V products of pairs j
+// (and j + 1, in groups of two) that read them. The P.V product reads P from TMEM. (On this part an M=128,
+// K=16 MMA costs about the same for N = 64 and N = 128, so 128-key chunks halve the cost of the score
+// products.)
 //
 // CTA layout (384 threads, one CTA per SM, persistent):
 //   warp 0      K loader: 128-row chunks into a ring of NST stages, per-item sample list; publishes each
@@ -35,7 +37,8 @@
 //               keeps the running max and sum, rescales O only when the running max grows by more than 2^8,
 //               and runs the epilogue.
 // Loaders copy with cp.async and arrive on the stage barrier when their copies complete.
-// TMEM (512 columns): S ring at [0, 128 R); O of tile t at [128 R + d t, 128 R + d (t + 1)).
+// TMEM (512 columns): S ring at [0, 256); d = 64: P of tile t at [256 + 64 t, 320 + 64 t), O of tile t at
+// [384 + 64 t, 448 + 64 t); d = 128: O of tile t at [256 + 128 t, 384 + 128 t).
 // Every mbarrier wait is bounded; on expiry the kernel sets the status bit, the other warps give up, the
 // loaders wait for their copies, the MMA issuer drains the tensor core, and TMEM is freed before exit.
 #include <math.h>

@@ -39,7 +39,7 @@ TRAFFIC = {
     # by the rows processed: attention 205.9 MB read + 46.8 MB written per 4-head launch; hash 134.2 + 6.2 MB.
     ("attn", "long_bf16_n131072", "tc"): {
         "file": "ha_attn_tc.cu",
-        "sha256": "d9bd25d08f1e6b2b71ae95ff389b4a01e5ccbdd43cd0f50bca7f8586108e97bc",
+        "sha256": "a84a9f305c2ab9e21b2b7e7f88f78aa375e948dc8162dfa1f90f93b6c2f84901",
         "bytes": 8 * (205_855_232 + 46_793_728)},
     ("hash", "long_bf16_n131072", "tc"): {
         "file": "ha_hash.cu",

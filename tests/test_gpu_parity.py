@@ -100,6 +100,8 @@ CASES = [
     ("all_sampled", 1024, 64, 1, 64, 1024, 6, False, 0, "bf16"),
     ("r16_two_pass", 4096, 64, 2, 256, 128, 16, False, 0, "bf16"),
     ("r12_two_pass", 2048, 128, 1, 128, 64, 12, False, 0, "fp32"),
+    ("r10_one_pass", 4096, 64, 2, 256, 64, 10, False, 0, "bf16"),    # 1024-way digit: large scatter stage
+    ("r9_one_pass", 2048, 128, 2, 128, 64, 9, False, 0, "bf16"),
     ("causal_small", 4096, 64, 2, 128, 64, 6, True, 512, "bf16"),
     ("causal_d128", 8192, 128, 2, 256, 128, 7, True, 1024, "bf16"),
     ("causal_exact_only", 1024, 64, 2, 64, 32, 6, True, 4096, "bf16"),

@@ -24,7 +24,7 @@ EXPORTS = [
     "hyper_attn_forward_host", "hyper_attn_draw", "hyper_attn_levels", "hyper_attn_debug_copy",
     "hyper_attn_status", "hyper_attn_last_launch_count", "hyper_attn_last_error", "hyper_attn_destroy",
     "hyper_attn_version", "hyper_attn_profile", "hyper_attn_profile_read",
-    "hyper_attn_last_kernel", "hyper_attn_forward_noalloc",
+    "hyper_attn_last_kernel", "hyper_attn_forward_noalloc", "hyper_attn_exact",
 ]
 KERNEL_CLASSES = ["hash", "sort", "attn", "causal_base"]
 
@@ -66,6 +66,7 @@ def lib():
     fwd = [vp, vp, vp, vp, vp, i64, ci, ci, ci, ci, ci, ci, u64]
     L.hyper_attn_forward.argtypes = fwd
     L.hyper_attn_forward_host.argtypes = fwd
+    L.hyper_attn_exact.argtypes = [vp, vp, vp, vp, vp, i64, ci, ci, ci]
     L.hyper_attn_draw.argtypes = [u64, ci, ci, i64, i64, ci, ci, i64, vp, vp]
     L.hyper_attn_levels.argtypes = [i64, ci, i64, ctypes.POINTER(ci), ctypes.POINTER(i64)]
     L.hyper_attn_debug_copy.argtypes = [vp, ci, ci, vp, ctypes.c_size_t]
@@ -153,6 +154,10 @@ class HyperAttention:
         """Device tensors (torch CUDA tensors or raw device addresses)."""
         self._check(lib().hyper_attn_forward(self._h, _ptr(Q), _ptr(K), _ptr(V), _ptr(O), n, d, heads, block, m, r,
                                              int(causal), seed))
+
+    def exact(self, Q, K, V, O, *, n, d, heads, causal):
+        """Exact softmax attention (device tensors) on the tensor-core kernel; enqueued on the handle's stream."""
+        self._check(lib().hyper_attn_exact(self._h, _ptr(Q), _ptr(K), _ptr(V), _ptr(O), n, d, heads, int(causal)))
 
     def forward_host(self, Q, K, V, O, *, n, d, heads, block, m, r, causal, seed):
         """Host buffers (numpy arrays or CPU torch tensors, preferably page-locked); blocks until O is ready."""

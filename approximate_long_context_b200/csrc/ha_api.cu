@@ -515,6 +515,31 @@ int hyper_attn_forward(hyper_attn_t h, const void *Q, const void *K, const void 
     return run_forward(h, Q, K, V, O, s, seed, h->opt.bh_offset);
 }
 
+int hyper_attn_exact(hyper_attn_t h, const void *Q, const void *K, const void *V, void *O, int64_t n, int d,
+                     int heads, int causal) {
+    if (!h) return HA_ERR_INVALID_ARG;
+    h->err.clear();
+    int rc = check_ptrs(h, Q, K, V, O);
+    if (rc) return rc;
+    if (heads <= 0 || n <= 0) return fail(h, HA_ERR_INVALID_ARG, "heads and n must be positive");
+    if (causal != 0 && causal != 1) return fail(h, HA_ERR_INVALID_ARG, "causal must be 0 or 1");
+    if (d != 64 && d != 128) return fail(h, HA_ERR_UNSUPPORTED, "d must be 64 or 128");
+    if (h->opt.dtype != HA_DTYPE_BF16) return fail(h, HA_ERR_UNSUPPORTED, "exact attention needs bf16 inputs");
+    if (n % 128 != 0) return fail(h, HA_ERR_UNSUPPORTED, "exact attention needs n to be a multiple of 128");
+    DeviceGuard g(h->device);
+    rc = ensure_workspace(h, 256);   // the status word (first 256 bytes of every layout)
+    if (rc) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(h->opt.stream);
+    const int out_dtype = h->opt.out_dtype < 0 ? h->opt.dtype : h->opt.out_dtype;
+    const int k = ha::launch_exact_tc(Q, K, V, h->opt.batch * heads, n, d, causal, O, out_dtype,
+                                      reinterpret_cast<int *>(h->ws + h->lay.status), st);
+    if (k == -2) return fail(h, HA_ERR_UNSUPPORTED, "shape not supported by the exact kernel");
+    if (k < 0) return fail(h, HA_ERR_CUDA, "exact attention launch failed: %s", cudaGetErrorString(cudaGetLastError()));
+    h->last_launches = k;
+    h->last_kernel = HA_KERNEL_TC;
+    return HA_OK;
+}
+
 int hyper_attn_forward_host(hyper_attn_t h, const void *Q, const void *K, const void *V, void *O, int64_t n, int d,
                             int heads, int block, int m, int r, int causal, uint64_t seed) {
     if (!h) return HA_ERR_INVALID_ARG;

@@ -61,7 +61,9 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleLog2 = 8.0f;   // rescale O only when the running max grows by more than this
 
-enum { MODE_LEVEL = 0, MODE_CAUSAL = 1 };
+// MODE_DENSE: exact (non-causal) softmax attention of every query tile against every key chunk of its
+// sequence, with the CAUSAL mode's work layout (a "leaf" is the whole sequence) and no mask.
+enum { MODE_LEVEL = 0, MODE_CAUSAL = 1, MODE_DENSE = 2 };
 
 struct TcArgs {
     int mode;
@@ -135,8 +137,8 @@ __device__ __forceinline__ Item decode(const TcArgs &a, int64_t it64) {
         x.gt1 = pair * 2 + 1;
         x.v0 = x.gt0 < a.tiles_per_leaf;
         x.v1 = x.gt1 < a.tiles_per_leaf;
-        x.nc0 = x.v0 ? x.gt0 + 1 : 0;
-        x.nc1 = x.v1 ? x.gt1 + 1 : 0;
+        x.nc0 = x.v0 ? (MODE == MODE_DENSE ? a.tiles_per_leaf : x.gt0 + 1) : 0;
+        x.nc1 = x.v1 ? (MODE == MODE_DENSE ? a.tiles_per_leaf : x.gt1 + 1) : 0;
     }
     x.nc_max = max(x.nc0, x.nc1);
     x.npairs = x.nc0 + x.nc1;
@@ -823,7 +825,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                         w2 = a.lw2;
                     }
                 } else {
-                    bound = my_gt * 128 + r - c * kKC;
+                    bound = MODE == MODE_DENSE ? kKC - 1 : my_gt * 128 + r - c * kKC;
                 }
                 tc_fence_after();
                 const bool masked = __any_sync(0xffffffffu, bound < kKC - 1);
@@ -1056,9 +1058,15 @@ int launch_tc(const void *Q, const void *K, const void *V, TcArgs args, cudaStre
 
 int dispatch(int d, const void *Q, const void *K, const void *V, const TcArgs &args, cudaStream_t st) {
     const bool level = args.mode == MODE_LEVEL;
-    if (d == 64) return level ? launch_tc<64, MODE_LEVEL>(Q, K, V, args, st) : launch_tc<64, MODE_CAUSAL>(Q, K, V, args, st);
-    if (d == 128)
-        return level ? launch_tc<128, MODE_LEVEL>(Q, K, V, args, st) : launch_tc<128, MODE_CAUSAL>(Q, K, V, args, st);
+    const bool dense = args.mode == MODE_DENSE;
+    if (d == 64) {
+        if (level) return launch_tc<64, MODE_LEVEL>(Q, K, V, args, st);
+        return dense ? launch_tc<64, MODE_DENSE>(Q, K, V, args, st) : launch_tc<64, MODE_CAUSAL>(Q, K, V, args, st);
+    }
+    if (d == 128) {
+        if (level) return launch_tc<128, MODE_LEVEL>(Q, K, V, args, st);
+        return dense ? launch_tc<128, MODE_DENSE>(Q, K, V, args, st) : launch_tc<128, MODE_CAUSAL>(Q, K, V, args, st);
+    }
     return -2;
 }
 
@@ -1119,6 +1127,27 @@ int launch_causal_base_tc(const void *Q, const void *K, const void *V, int64_t b
     a.status = status;
     a.items = bh * a.nleaves * a.pairs_per_leaf;
     a.per_outer = static_cast<uint32_t>(bh * a.nleaves);
+    if (a.items >= (int64_t(1) << 31)) return -2;
+    return dispatch(d, Q, K, V, a, st);
+}
+
+int launch_exact_tc(const void *Q, const void *K, const void *V, int64_t bh, int64_t n, int d, int causal, void *O,
+                    int out_dtype, int *status, cudaStream_t st) {
+    if ((d != 64 && d != 128) || n <= 0 || n % 128 != 0 || bh * n >= (int64_t(1) << 31)) return -2;
+    TcArgs a{};
+    a.mode = causal ? MODE_CAUSAL : MODE_DENSE;
+    a.n = n;
+    a.bh = bh;
+    a.leaf = n;
+    a.nleaves = 1;
+    a.levels = 0;
+    a.tiles_per_leaf = static_cast<int>(n / 128);
+    a.pairs_per_leaf = (a.tiles_per_leaf + 1) / 2;
+    a.O = O;
+    a.out_dtype = out_dtype;
+    a.status = status;
+    a.items = bh * a.pairs_per_leaf;
+    a.per_outer = static_cast<uint32_t>(bh);
     if (a.items >= (int64_t(1) << 31)) return -2;
     return dispatch(d, Q, K, V, a, st);
 }

@@ -66,6 +66,9 @@ int launch_attn_tc(const Level &lv, const void *Q, const void *K, const void *V,
 int launch_causal_base_tc(const void *Q, const void *K, const void *V, int64_t bh, int64_t n, int d,
                           int64_t leaf, int levels, const float *Opart, const float *Lpart,
                           void *O, int out_dtype, int *status, cudaStream_t st);
+// Exact softmax attention (causal: keys up to the query) of bh problems of n rows on the tensor cores.
+int launch_exact_tc(const void *Q, const void *K, const void *V, int64_t bh, int64_t n, int d, int causal, void *O,
+                    int out_dtype, int *status, cudaStream_t st);
 
 // ---- host-side draws (ha_draws.cpp) ----
 void draw_projection(uint64_t seed, int d, int r, float *P);

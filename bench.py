@@ -324,6 +324,28 @@ def run_ours(args, w: wl.Workload):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
     e2e_value = units / (e2e_ms * 1e-3) / 1e6
 
+    # same-box comparison with exact softmax attention (the tensor-core exact kernel) on the same inputs
+    vs_exact = None
+    if not args.no_exact and w.dtype == "bf16" and w.n % 128 == 0:
+        O2 = torch.empty_like(O)
+        ha.set_options(dtype=w.dtype, batch=w.batch, causal_base=w.base or 4096, stream=stream.cuda_stream,
+                       kernel=args.kernel, bh_offset=sh.offset)
+        ha.exact(Q, K, V, O2, n=w.n, d=w.d, heads=w.heads, causal=w.causal)   # warm-up
+        x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        x0.record(stream)
+        for _ in range(2):
+            ha.exact(Q, K, V, O2, n=w.n, d=w.d, heads=w.heads, causal=w.causal)
+        x1.record(stream)
+        torch.cuda.synchronize(dev)
+        assert ha.status() == 0, ha.last_error()
+        ex_ms = x0.elapsed_time(x1) / 2
+        ex_flops = w.bh * 4.0 * w.n * w.n * w.d * (0.5 if w.causal else 1.0)
+        vs_exact = {"exact_ms_per_step": ex_ms, "speedup": ex_ms / ms_max,
+                    "exact_tflops": ex_flops / (ex_ms * 1e-3) / 1e12, "exact_kernel": "tcgen05",
+                    "note": "exact softmax attention on the same inputs and GPU; causal counts half the pairs"}
+        del O2
+
     # roofline of the dominant kernel class; sort and attention launch once per level
     peaks, peak_src = load_peaks()
     family = ha.last_kernel()
@@ -384,6 +406,7 @@ def run_ours(args, w: wl.Workload):
             "clocks": clk.summary(),
             "cpu_baseline": cpu,
             "approx_error": err,
+            "vs_exact": vs_exact,
         }
         print(json.dumps(line), flush=True)
     ha.close()
@@ -403,6 +426,7 @@ def main():
     ap.add_argument("--heads", type=int, default=0,
                     help="run the workload with this many heads instead of its own (small profiler captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-exact", action="store_true", help="skip the same-box exact-attention comparison")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

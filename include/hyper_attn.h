@@ -101,6 +101,19 @@ HA_API int hyper_attn_forward(hyper_attn_t h, const void *Q, const void *K, cons
                        int64_t n, int d, int heads, int block, int m, int r, int causal, uint64_t seed);
 
 /*
+ * Exact softmax attention O = softmax(Q K^T) V for every (batch, head) problem: no sampling, hashing or
+ * blocks; causal = 1 lets query i see keys 0..i. This is the reference the approximation is measured
+ * against ("HyperAttention: Long-context Attention in Near-Linear Time", research-map summary, "Key
+ * results": speed-ups are quoted against exact attention), computed here on the same tensor-core kernel
+ * as the method's exact causal leaves. Arguments as for hyper_attn_forward (device pointers, the
+ * handle's dtype, batch, out_dtype and stream), with these limits: bf16 inputs, d in {64, 128}, n a
+ * multiple of 128 (HA_ERR_UNSUPPORTED otherwise). Enqueued on the handle's stream; device-side wait
+ * timeouts surface through hyper_attn_status.
+ */
+HA_API int hyper_attn_exact(hyper_attn_t h, const void *Q, const void *K, const void *V, void *O,
+                            int64_t n, int d, int heads, int causal);
+
+/*
  * Same computation with HOST buffers: copies Q, K, V to handle-owned device buffers, runs the forward
  * pass, copies O back and waits. Returns when O is valid on the host. The (batch, head) problems go
  * through in up to 8 contiguous groups so that host-to-device copies, the forward pass (on the handle's

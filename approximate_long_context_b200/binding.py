@@ -45,6 +45,7 @@ class Options(ctypes.Structure):
         ("kernel", ctypes.c_int),
         ("debug_captures", ctypes.c_int),
         ("bh_offset", ctypes.c_int64),
+        ("test_stall_ms", ctypes.c_int),
     ]
 
 
@@ -137,7 +138,7 @@ class HyperAttention:
             raise HAError(rc, lib().hyper_attn_last_error(self._h).decode())
 
     def set_options(self, *, dtype="bf16", out_dtype=None, batch=1, causal_base=4096, stream=None,
-                    kernel="auto", debug_captures=False, bh_offset=0):
+                    kernel="auto", debug_captures=False, bh_offset=0, test_stall_ms=0):
         o = Options()
         o.dtype = DTYPES[dtype]
         o.out_dtype = -1 if out_dtype is None else DTYPES[out_dtype]
@@ -147,6 +148,7 @@ class HyperAttention:
         o.kernel = KERNELS[kernel]
         o.debug_captures = int(bool(debug_captures))
         o.bh_offset = bh_offset
+        o.test_stall_ms = test_stall_ms
         self._check(lib().hyper_attn_set_options(self._h, ctypes.byref(o)))
         self.options = o
 

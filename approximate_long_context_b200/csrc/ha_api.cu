@@ -334,6 +334,7 @@ int run_forward(hyper_attn_t h, const void *Q, const void *K, const void *V, voi
     float *Opart = reinterpret_cast<float *>(ws + lay.Opart);
     float *Lpart = reinterpret_cast<float *>(ws + lay.Lpart);
     int *status = reinterpret_cast<int *>(ws + lay.status);
+    const int64_t stall_ns = static_cast<int64_t>(h->opt.test_stall_ms) * 1000000;   // test hook, 0 = off
     const size_t half_rows = static_cast<size_t>(s.bh) * (s.n / 2);
 
     int launches = 0;
@@ -398,7 +399,7 @@ int run_forward(hyper_attn_t h, const void *Q, const void *K, const void *V, voi
         ev = prof_begin();
         if (use_tc) family = HA_KERNEL_TC;
         if (use_tc) k = ha::launch_attn_tc(lv, Q, K, V, s.d, perm, inv, S, s.m, s.nodes_total, O, out_dtype, lse, Op,
-                                           Lp, status, st);
+                                           Lp, status, st, stall_ns);
         if (k == -2 && h->opt.kernel != HA_KERNEL_TC) family = HA_KERNEL_SIMT;
         if (k == -2 && h->opt.kernel != HA_KERNEL_TC)
             k = ha::launch_attn_simt(lv, Q, K, V, dtype, s.d, perm, inv, S, s.m, s.nodes_total, O, out_dtype, lse, Op,
@@ -411,7 +412,7 @@ int run_forward(hyper_attn_t h, const void *Q, const void *K, const void *V, voi
         ev = prof_begin();
         if (use_tc && family != HA_KERNEL_SIMT) family = HA_KERNEL_TC;
         if (use_tc) k = ha::launch_causal_base_tc(Q, K, V, s.bh, s.n, s.d, s.leaf, s.levels, Opart, Lpart, O, out_dtype,
-                                                  status, st);
+                                                  status, st, stall_ns);
         if (k == -2 && h->opt.kernel != HA_KERNEL_TC) family = HA_KERNEL_SIMT;
         if (k == -2 && h->opt.kernel != HA_KERNEL_TC)
             k = ha::launch_causal_base_simt(Q, K, V, dtype, s.bh, s.n, s.d, s.leaf, s.levels, Opart, Lpart, O,
@@ -434,6 +435,7 @@ int validate_options(hyper_attn_t h, const ha_options *o) {
     if (o->debug_captures != 0 && o->debug_captures != 1) return fail(h, HA_ERR_INVALID_ARG, "bad debug_captures");
     if (o->bh_offset < 0 || o->bh_offset > (int64_t(1) << 40))
         return fail(h, HA_ERR_INVALID_ARG, "bh_offset out of range");
+    if (o->test_stall_ms < 0 || o->test_stall_ms > 1000) return fail(h, HA_ERR_INVALID_ARG, "test_stall_ms out of range");
     return HA_OK;
 }
 
@@ -459,6 +461,7 @@ void hyper_attn_default_options(ha_options *o) {
     o->kernel = HA_KERNEL_AUTO;
     o->debug_captures = 0;
     o->bh_offset = 0;
+    o->test_stall_ms = 0;
 }
 
 int hyper_attn_version(void) { return kVersion; }

@@ -86,6 +86,7 @@ struct TcArgs {
     int out_dtype;
     float *lse, *Opart_w, *Lpart_w;
     int *status;
+    int64_t stall_ns;      // test hook: > 0 makes the first softmax wait give up after this long (see bNever)
     int64_t items;
     uint32_t per_outer;    // LEVEL: items per problem; CAUSAL: items per query-tile pair index
 };
@@ -204,7 +205,7 @@ struct Cfg {
                          bSFull = bRowsFull + NST,
                          bPFull = bSFull + R, bPVDone = bPFull + R, bPVDoneT = bPVDone + R, bOFree = bPVDoneT + 4,
                          bDrain = bOFree + 2, bQStage = bDrain + 2, bSFree = bQStage + 2 * QB, bPFullT = bSFree + R,
-                         kNumBars = bPFullT + 2;
+                         bNever = bPFullT + 2, kNumBars = bNever + 1;
     static constexpr int kTmemSlot = kBars + kNumBars * 8;
     static constexpr int kAbort = kTmemSlot + 4;
     static constexpr int kBytes = kAbort + 4;
@@ -322,6 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
         for (int b = 0; b < C::R; ++b) mbar_init(bar(C::bPVDone + b), 1);
         for (int i = 0; i < 4; ++i) mbar_init(bar(C::bPVDoneT + i), 1);
         for (int t = 0; t < 2; ++t) mbar_init(bar(C::bPFullT + t), 128);   // kSepP: P of a tile's pair written
+        mbar_init(bar(C::bNever), 1);              // nothing arrives: the test hook's wait never completes
         for (int t = 0; t < 2; ++t) {
             mbar_init(bar(C::bDrain + t), 1);
             mbar_init(bar(C::bOFree + t), 128);
@@ -812,6 +814,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                 const uint32_t k = kp + static_cast<uint32_t>(pair_index(x, t, c));
                 const int buf = static_cast<int>(k % C::R);
                 const uint32_t tS = trow + buf * 128;
+                if (a.stall_ns > 0 && it == first && c == 0 &&
+                    !mbar_wait(bar(C::bNever), 0, abort_flag, static_cast<uint64_t>(a.stall_ns))) {
+                    ok = false;   // test hook: this wait runs out, sets the abort flag, and every role stops
+                    break;
+                }
                 if (!mbar_wait(bar(C::bSFull + buf), (k / C::R) & 1, abort_flag)) { ok = false; break; }
                 // column bound: columns > bound are masked (bound >= 127: none)
                 int bound = kKC - 1;
@@ -1074,7 +1081,7 @@ int dispatch(int d, const void *Q, const void *K, const void *V, const TcArgs &a
 
 int launch_attn_tc(const Level &lv, const void *Q, const void *K, const void *V, int d, const int32_t *perm,
                    const int32_t *inv, const int32_t *S, int m, int64_t nodes_total, void *O, int out_dtype,
-                   float *lse, float *Opart, float *Lpart, int *status, cudaStream_t st) {
+                   float *lse, float *Opart, float *Lpart, int *status, cudaStream_t st, int64_t stall_ns) {
     if ((d != 64 && d != 128) || lv.bp % 128 != 0 || lv.bp > kMaxBlock || m > kMaxSampleList ||
         lv.bh * lv.n >= (int64_t(1) << 31))
         return -2;
@@ -1099,6 +1106,7 @@ int launch_attn_tc(const Level &lv, const void *Q, const void *K, const void *V,
     a.Opart_w = Opart;
     a.Lpart_w = Lpart;
     a.status = status;
+    a.stall_ns = stall_ns;
     a.items = lv.bh * lv.nodes * (lv.seg_len / lv.bp) * a.pairs_per_block;
     a.per_outer = static_cast<uint32_t>((lv.seg_len / lv.bp) * a.pairs_per_block);
     if (a.items >= (int64_t(1) << 31)) return -2;
@@ -1107,7 +1115,7 @@ int launch_attn_tc(const Level &lv, const void *Q, const void *K, const void *V,
 
 int launch_causal_base_tc(const void *Q, const void *K, const void *V, int64_t bh, int64_t n, int d, int64_t leaf,
                           int levels, const float *Opart, const float *Lpart, void *O, int out_dtype, int *status,
-                          cudaStream_t st) {
+                          cudaStream_t st, int64_t stall_ns) {
     if ((d != 64 && d != 128) || leaf % 128 != 0 || n % leaf != 0 || levels > kMaxLevels ||
         bh * n >= (int64_t(1) << 31) || static_cast<int64_t>(levels) * bh * (n / 2) >= (int64_t(1) << 32))
         return -2;
@@ -1125,6 +1133,7 @@ int launch_causal_base_tc(const void *Q, const void *K, const void *V, int64_t b
     a.O = O;
     a.out_dtype = out_dtype;
     a.status = status;
+    a.stall_ns = stall_ns;
     a.items = bh * a.nleaves * a.pairs_per_leaf;
     a.per_outer = static_cast<uint32_t>(bh * a.nleaves);
     if (a.items >= (int64_t(1) << 31)) return -2;
@@ -1146,6 +1155,7 @@ int launch_exact_tc(const void *Q, const void *K, const void *V, int64_t bh, int
     a.O = O;
     a.out_dtype = out_dtype;
     a.status = status;
+    a.stall_ns = 0;
     a.items = bh * a.pairs_per_leaf;
     a.per_outer = static_cast<uint32_t>(bh);
     if (a.items >= (int64_t(1) << 31)) return -2;

@@ -62,10 +62,12 @@ int launch_causal_base_simt(const void *Q, const void *K, const void *V, int dty
 // Tensor-core (tcgen05) kernels; return -2 when a shape is not supported by the tensor-core path.
 int launch_attn_tc(const Level &lv, const void *Q, const void *K, const void *V, int d,
                    const int32_t *perm, const int32_t *inv, const int32_t *S, int m, int64_t nodes_total,
-                   void *O, int out_dtype, float *lse, float *Opart, float *Lpart, int *status, cudaStream_t st);
+                   void *O, int out_dtype, float *lse, float *Opart, float *Lpart, int *status, cudaStream_t st,
+                   int64_t stall_ns = 0);
 int launch_causal_base_tc(const void *Q, const void *K, const void *V, int64_t bh, int64_t n, int d,
                           int64_t leaf, int levels, const float *Opart, const float *Lpart,
-                          void *O, int out_dtype, int *status, cudaStream_t st);
+                          void *O, int out_dtype, int *status, cudaStream_t st, int64_t stall_ns = 0);
+// stall_ns > 0 (test hook): the first softmax wait gives up after stall_ns on a barrier nothing completes.
 // Exact softmax attention (causal: keys up to the query) of bh problems of n rows on the tensor cores.
 int launch_exact_tc(const void *Q, const void *K, const void *V, int64_t bh, int64_t n, int d, int causal, void *O,
                     int out_dtype, int *status, cudaStream_t st);

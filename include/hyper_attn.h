@@ -69,6 +69,11 @@ typedef struct {
                              of local problem i are those of problem bh_offset + i, so a run split over
                              several calls or GPUs (each taking a contiguous range of problems) gives the
                              same result as one call over all problems. Default 0. */
+    int test_stall_ms;    /* Test hook for the failure path, 0..1000. When > 0, the tensor-core attention
+                             kernel's first softmax wait targets a barrier that nothing ever completes and
+                             gives up after this many milliseconds: every role of the kernel then stops,
+                             the output is undefined, and hyper_attn_status reports HA_ERR_TIMEOUT. The
+                             device stays usable. Default 0 (off). */
 } ha_options;
 
 /* Create a handle bound to CUDA device `device`. The handle owns a grow-only device workspace (ranks,

@@ -65,6 +65,10 @@ def _load():
     lib.ora_exact_attention.argtypes = [_f32p, _f32p, _f32p, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
                                         vp, ctypes.c_int64, _f64p]
     lib.ora_exact_attention.restype = ctypes.c_int
+    lib.ora_diagnostics.argtypes = [_f32p, _f32p, ctypes.c_int64, ctypes.c_int, ctypes.c_int64, ctypes.c_int,
+                                    ctypes.c_uint64, ctypes.c_int64, ctypes.POINTER(ctypes.c_double),
+                                    ctypes.POINTER(ctypes.c_double)]
+    lib.ora_diagnostics.restype = ctypes.c_int
     lib.ora_num_threads.argtypes = []
     lib.ora_num_threads.restype = ctypes.c_int
     _lib = lib
@@ -161,6 +165,18 @@ def forward(Q, K, V, *, block: int, m: int, r: int, causal: bool, seed: int, bh:
         out["L1"] = L1[:nsel]
         out["L2"] = L2[:nsel]
     return out
+
+
+def diagnostics(Q, K, *, block: int, r: int, seed: int, first_col: int = 0):
+    """(alpha, kappa) of one non-causal problem: alpha = n * max_{j >= first_col} ||(D^-1 A) e_j||^2 and kappa =
+    max/min over rows of the row sums of A outside the row's sortLSH block (see oracle.c for the readings)."""
+    Q = np.ascontiguousarray(Q, np.float32)
+    K = np.ascontiguousarray(K, np.float32)
+    n, d = Q.shape
+    alpha, kappa = ctypes.c_double(), ctypes.c_double()
+    _check(_load().ora_diagnostics(Q, K, n, d, block, r, seed, first_col, ctypes.byref(alpha), ctypes.byref(kappa)),
+           "diagnostics")
+    return alpha.value, kappa.value
 
 
 def exact_attention(Q, K, V, *, causal: bool, rows=None) -> np.ndarray:

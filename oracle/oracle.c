@@ -533,6 +533,76 @@ int ora_exact_attention(const float *Q, const float *K, const float *V, int64_t 
     return ORA_OK;
 }
 
+/* Hardness diagnostics of one (non-causal) problem ("HyperAttention: Long-context Attention in Near-Linear
+ * Time", research-map summary, "Approach", "Key results", "Limitations", and the abstract page: the guarantee
+ * rests on the max column norm of the normalised attention matrix D^-1 A and on the ratio of row norms of A
+ * once its large entries are removed).
+ * READING (alpha): alpha = n * max_{j >= first_col} sum_i W_ij^2 with W = D^-1 A, A_ij = exp(q_i . k_j); it is
+ *   1 for uniform attention and n^2 when every row puts all its weight on one column. first_col > 0 drops the
+ *   first columns (the pages drop 32 sink-like columns for one model).
+ * READING (kappa): the large entries are the ones the method computes exactly, i.e. the aligned blocks of the
+ *   sortLSH order (block b' = min(block, n), ranks from this oracle's hash, stable sort). Row norm = row sum
+ *   (the quantity the normaliser estimate needs). kappa = max_i R_i / min_i R_i with R_i = sum of A_ij over
+ *   the columns outside row i's block; 0/0 gives NaN and x/0 gives +inf.
+ * Everything in double precision, in the order of the definitions. */
+int ora_diagnostics(const float *Q, const float *K, int64_t n, int d, int64_t block, int r, uint64_t seed,
+                    int64_t first_col, double *alpha_out, double *kappa_out)
+{
+    if (n <= 0 || d <= 0 || block <= 0 || r < 0 || r > 16 || first_col < 0 || first_col >= n) return ORA_EINVAL;
+    const int64_t bp = block < n ? block : n;
+    float *P = (float *)malloc(sizeof(float) * (size_t)(d * (r > 0 ? r : 1)));
+    uint16_t *rq = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)n), *rk = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)n);
+    uint8_t *fl = (uint8_t *)malloc((size_t)n);
+    int32_t *pq = (int32_t *)malloc(sizeof(int32_t) * (size_t)n), *pk = (int32_t *)malloc(sizeof(int32_t) * (size_t)n);
+    int64_t *posq = (int64_t *)malloc(sizeof(int64_t) * (size_t)n), *posk = (int64_t *)malloc(sizeof(int64_t) * (size_t)n);
+    double *m = (double *)malloc(sizeof(double) * (size_t)n), *D = (double *)malloc(sizeof(double) * (size_t)n);
+    double *logR = (double *)malloc(sizeof(double) * (size_t)n), *col = (double *)calloc((size_t)n, sizeof(double));
+    if (!P || !rq || !rk || !fl || !pq || !pk || !posq || !posk || !m || !D || !logR || !col) return ORA_ENOMEM;
+    if (r > 0) ora_draw_projection(seed, d, r, P);
+    ora_hash_rows(Q, n, d, P, r, rq, fl);
+    ora_hash_rows(K, n, d, P, r, rk, fl);
+    ora_sort_segment(rq, n, pq);
+    ora_sort_segment(rk, n, pk);
+    for (int64_t p = 0; p < n; ++p) { posq[pq[p]] = p; posk[pk[p]] = p; }
+    /* rows: max, normaliser, and the sum outside the row's block (all shifted by the row max) */
+    for (int64_t i = 0; i < n; ++i) {
+        double mx = -INFINITY;
+        for (int64_t j = 0; j < n; ++j) {
+            double s = dot_fd(Q + i * d, K + j * d, d);
+            if (s > mx) mx = s;
+        }
+        double den = 0.0, rest = 0.0;
+        for (int64_t j = 0; j < n; ++j) {
+            double e = exp(dot_fd(Q + i * d, K + j * d, d) - mx);
+            den += e;
+            if (posk[j] / bp != posq[i] / bp) rest += e;
+        }
+        m[i] = mx;
+        D[i] = den;
+        logR[i] = rest > 0.0 ? log(rest) + mx : -INFINITY;
+    }
+    /* columns: squared norms of W = D^-1 A */
+    for (int64_t i = 0; i < n; ++i)
+        for (int64_t j = 0; j < n; ++j) {
+            double w = exp(dot_fd(Q + i * d, K + j * d, d) - m[i]) / D[i];
+            col[j] += w * w;
+        }
+    double cmax = 0.0;
+    for (int64_t j = first_col; j < n; ++j) if (col[j] > cmax) cmax = col[j];
+    *alpha_out = (double)n * cmax;
+    double lo = INFINITY, hi = -INFINITY;
+    for (int64_t i = 0; i < n; ++i) {
+        if (logR[i] < lo) lo = logR[i];
+        if (logR[i] > hi) hi = logR[i];
+    }
+    if (hi == -INFINITY) *kappa_out = NAN;              /* every row: nothing outside its block */
+    else if (lo == -INFINITY) *kappa_out = INFINITY;    /* some rows have nothing outside their block */
+    else *kappa_out = exp(hi - lo);
+    free(P); free(rq); free(rk); free(fl); free(pq); free(pk); free(posq); free(posk);
+    free(m); free(D); free(logR); free(col);
+    return ORA_OK;
+}
+
 int ora_num_threads(void)
 {
 #ifdef _OPENMP

@@ -334,3 +334,62 @@ def test_level_perms(ora):
         s = j * 256
         assert np.array_equal(pq[j * 128:(j + 1) * 128], np.argsort(rank[s + 128:s + 256], kind="stable"))
         assert np.array_equal(pk[j * 128:(j + 1) * 128], np.argsort(rank[n + s:n + s + 128], kind="stable"))
+
+
+# ---------------------------------------------------------------------------------------- hardness diagnostics
+# alpha = n * max_j ||(D^-1 A) e_j||^2 and kappa = max/min row sum of A outside the row's sortLSH block
+# ("HyperAttention: Long-context Attention in Near-Linear Time", research-map summary, "Approach", "Key results").
+
+def test_diagnostics_uniform_attention(ora):
+    """Q = 0: every softmax row is uniform, so each column has squared norm n * (1/n)^2 and alpha = 1; every row
+    has the same n - b' unit entries outside its block, so kappa = 1. With one block, nothing is outside: NaN."""
+    rng = np.random.default_rng(41)
+    n, d = 96, 16
+    Q = np.zeros((n, d), np.float32)
+    K = rng.standard_normal((n, d)).astype(np.float32)
+    alpha, kappa = ora.diagnostics(Q, K, block=32, r=5, seed=3)
+    assert alpha == pytest.approx(1.0, rel=1e-12)
+    assert kappa == pytest.approx(1.0, rel=1e-12)
+    alpha1, kappa1 = ora.diagnostics(Q, K, block=n, r=5, seed=3)
+    assert alpha1 == pytest.approx(1.0, rel=1e-12) and np.isnan(kappa1)
+
+
+def test_diagnostics_dominant_column(ora):
+    """One key aligned with every query and far larger than the rest takes almost all of every row's weight:
+    alpha -> n^2. Dropping that column (first_col past it) leaves alpha far below."""
+    rng = np.random.default_rng(43)
+    n, d = 64, 16
+    u = rng.standard_normal(d).astype(np.float32)
+    u /= np.linalg.norm(u)
+    Q = (np.tile(u, (n, 1)) * 4.0 + 0.01 * rng.standard_normal((n, d))).astype(np.float32)
+    K = (0.1 * rng.standard_normal((n, d))).astype(np.float32)
+    K[0] = 8.0 * u
+    alpha, _ = ora.diagnostics(Q, K, block=16, r=4, seed=5)
+    assert alpha == pytest.approx(n * n, rel=1e-6)
+    alpha_rest, _ = ora.diagnostics(Q, K, block=16, r=4, seed=5, first_col=1)
+    assert alpha_rest < 1e-6
+
+
+def test_diagnostics_kappa_planted_ratio(ora):
+    """All keys equal (k = u): a query row's entries are all exp(q . u). Half the queries are 0 (entries 1), half
+    are t*u (entries exp(t |u|^2)); every row has n - b' entries outside its block whatever the sort does, so
+    kappa = exp(t |u|^2) exactly."""
+    n, d, t = 128, 8, 0.75
+    u = np.linspace(-1.0, 1.0, d).astype(np.float32)
+    K = np.tile(u, (n, 1)).astype(np.float32)
+    Q = np.zeros((n, d), np.float32)
+    Q[n // 2:] = (t * u).astype(np.float32)
+    _, kappa = ora.diagnostics(Q, K, block=32, r=6, seed=9)
+    s = float(np.dot((t * u).astype(np.float32).astype(np.float64), u.astype(np.float64)))
+    assert kappa == pytest.approx(np.exp(s), rel=1e-12)
+
+
+def test_diagnostics_alpha_ignores_row_order(ora):
+    """alpha depends on column norms of D^-1 A only: permuting the queries (rows) leaves it unchanged."""
+    rng = np.random.default_rng(47)
+    n, d = 80, 16
+    Q = (0.5 * rng.standard_normal((n, d))).astype(np.float32)
+    K = (0.5 * rng.standard_normal((n, d))).astype(np.float32)
+    a0, _ = ora.diagnostics(Q, K, block=16, r=5, seed=2)
+    a1, _ = ora.diagnostics(Q[rng.permutation(n)], K, block=16, r=5, seed=2)
+    assert a1 == pytest.approx(a0, rel=1e-12)

@@ -52,6 +52,7 @@ struct hyper_attn_s {
 namespace {
 
 constexpr int kVersion = 100;   // 0.1.0
+constexpr int kDiagMaxN = 16384;   // the diagnostics visit every entry of A
 
 size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
 
@@ -298,8 +299,9 @@ int upload_draws(hyper_attn_t h, uint64_t seed, const Shape &s, int64_t bh_offse
 }
 
 // The forward pass of shape s on device buffers; the problems' draws are keyed from global index bh_offset.
+// sort_only: stop after the hash and the sort (their outputs stay in the workspace; V and O are not used).
 int run_forward(hyper_attn_t h, const void *Q, const void *K, const void *V, void *O, const Shape &s,
-                uint64_t seed, int64_t bh_offset) {
+                uint64_t seed, int64_t bh_offset, bool sort_only = false) {
     cudaStream_t st = static_cast<cudaStream_t>(h->opt.stream);
     const int dtype = h->opt.dtype;
     const int out_dtype = h->opt.out_dtype < 0 ? dtype : h->opt.out_dtype;
@@ -393,6 +395,7 @@ int run_forward(hyper_attn_t h, const void *Q, const void *K, const void *V, voi
         }
         prof_end(ev, HA_KC_SORT, kl);
         if ((rc = count(kl, "sort"))) return rc;
+        if (sort_only) continue;
         float *Op = s.causal ? Opart + static_cast<size_t>(l - 1) * half_rows * s.d : nullptr;
         float *Lp = s.causal ? Lpart + static_cast<size_t>(l - 1) * half_rows : nullptr;
         int k = -2;
@@ -407,7 +410,7 @@ int run_forward(hyper_attn_t h, const void *Q, const void *K, const void *V, voi
         prof_end(ev, HA_KC_ATTN, k);
         if ((rc = count(k, "attention"))) return rc;
     }
-    if (s.causal) {
+    if (s.causal && !sort_only) {
         int k = -2;
         ev = prof_begin();
         if (use_tc && family != HA_KERNEL_SIMT) family = HA_KERNEL_TC;
@@ -516,6 +519,46 @@ int hyper_attn_forward(hyper_attn_t h, const void *Q, const void *K, const void 
     if (rc) return rc;
     DeviceGuard g(h->device);
     return run_forward(h, Q, K, V, O, s, seed, h->opt.bh_offset);
+}
+
+int hyper_attn_diagnostics(hyper_attn_t h, const void *Q, const void *K, int64_t n, int d, int heads, int block,
+                           int r, uint64_t seed, int64_t first_col, double *alpha, double *kappa) {
+    if (!h) return HA_ERR_INVALID_ARG;
+    h->err.clear();
+    if (!Q || !K || !alpha || !kappa) return fail(h, HA_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(Q) || !aligned16(K)) return fail(h, HA_ERR_INVALID_ARG, "Q and K must be 16-byte aligned");
+    if (heads <= 0) return fail(h, HA_ERR_INVALID_ARG, "heads must be positive");
+    if (n > kDiagMaxN) return fail(h, HA_ERR_INVALID_ARG, "diagnostics take n <= %d (every entry of A)", kDiagMaxN);
+    if (first_col < 0 || first_col >= n) return fail(h, HA_ERR_INVALID_ARG, "first_col must lie in [0, n)");
+    Shape s{};
+    int rc = check_shape(h, n, d, h->opt.batch * heads, block, 0, r, 0, &s);
+    if (rc) return rc;
+    DeviceGuard g(h->device);
+    cudaStream_t st = static_cast<cudaStream_t>(h->opt.stream);
+    const int esz = h->opt.dtype == HA_DTYPE_BF16 ? 2 : 4;
+    hyper_attn_s::Layout lay;
+    const size_t fwd_bytes = align_up(plan_layout(s, esz, h->opt.debug_captures, &lay));
+    const size_t diag_scratch = align_up(sizeof(float) * 4 * static_cast<size_t>(s.bh) * n);
+    const size_t diag_out = sizeof(double) * 2 * static_cast<size_t>(s.bh);
+    rc = ensure_workspace(h, fwd_bytes + diag_scratch + diag_out);   // the forward below reuses it as is
+    if (rc) return rc;
+    rc = run_forward(h, Q, K, nullptr, nullptr, s, seed, h->opt.bh_offset, true);
+    if (rc) return rc;
+    float *scratch = reinterpret_cast<float *>(h->ws + fwd_bytes);
+    double *out = reinterpret_cast<double *>(h->ws + fwd_bytes + diag_scratch);
+    const int32_t *inv = reinterpret_cast<const int32_t *>(h->ws + h->lay.inv[0]);
+    const int64_t bp = s.block < n ? s.block : n;
+    const int k = ha::launch_diagnostics(Q, K, h->opt.dtype == HA_DTYPE_BF16 ? 0 : 1, s.bh, n, d, inv, bp, first_col,
+                                         scratch, out, st);
+    if (k < 0) return fail(h, HA_ERR_CUDA, "diagnostics launch failed: %s", cudaGetErrorString(cudaGetLastError()));
+    std::vector<double> host(2 * static_cast<size_t>(s.bh));
+    HA_CUDA(h, cudaMemcpyAsync(host.data(), out, diag_out, cudaMemcpyDeviceToHost, st));
+    HA_CUDA(h, cudaStreamSynchronize(st));
+    for (int64_t b = 0; b < s.bh; ++b) {
+        alpha[b] = host[2 * b];
+        kappa[b] = host[2 * b + 1];
+    }
+    return HA_OK;
 }
 
 int hyper_attn_exact(hyper_attn_t h, const void *Q, const void *K, const void *V, void *O, int64_t n, int d,

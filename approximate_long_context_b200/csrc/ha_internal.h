@@ -72,6 +72,11 @@ int launch_causal_base_tc(const void *Q, const void *K, const void *V, int64_t b
 int launch_exact_tc(const void *Q, const void *K, const void *V, int64_t bh, int64_t n, int d, int causal, void *O,
                     int out_dtype, int *status, cudaStream_t st);
 
+// Hardness diagnostics (ha_diag.cu) of bh non-causal problems of n rows: out[2b] = alpha, out[2b+1] = kappa.
+// inv: level-0 inverse permutations [bh][2][n]; scratch: 4 * bh * n floats.
+int launch_diagnostics(const void *Q, const void *K, int dtype, int64_t bh, int64_t n, int d, const int32_t *inv,
+                       int64_t bp, int64_t first_col, float *scratch, double *out, cudaStream_t st);
+
 // ---- host-side draws (ha_draws.cpp) ----
 void draw_projection(uint64_t seed, int d, int r, float *P);
 int draw_samples(uint64_t seed, uint64_t bh, uint64_t node, int64_t N, int m, int32_t *S, uint8_t *scratch);

@@ -346,6 +346,21 @@ def run_ours(args, w: wl.Workload):
                     "note": "exact softmax attention on the same inputs and GPU; causal counts half the pairs"}
         del O2
 
+    # optional: hardness diagnostics on the first rows of head 0 (every entry of A is visited, so a slice)
+    diag = None
+    if args.diagnostics and rank == 0 and not w.causal:
+        nd = min(w.n, 4096)
+        Qs, Ks = Q[:1, :nd].contiguous(), K[:1, :nd].contiguous()
+        ha.set_options(dtype=w.dtype, batch=1, causal_base=w.base or 4096, stream=stream.cuda_stream, kernel=args.kernel)
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        a0, k0 = ha.diagnostics(Qs, Ks, n=nd, d=w.d, heads=1, block=w.block, r=w.r, seed=w.algo_seed)
+        g1.record(stream)
+        torch.cuda.synchronize(dev)
+        a32, _ = ha.diagnostics(Qs, Ks, n=nd, d=w.d, heads=1, block=w.block, r=w.r, seed=w.algo_seed, first_col=32)
+        diag = {"rows": nd, "head": 0, "alpha": float(a0[0]), "alpha_without_first_32": float(a32[0]),
+                "kappa": float(k0[0]), "ms": g0.elapsed_time(g1)}
+
     # roofline of the dominant kernel class; sort and attention launch once per level
     peaks, peak_src = load_peaks()
     family = ha.last_kernel()
@@ -408,6 +423,8 @@ def run_ours(args, w: wl.Workload):
             "approx_error": err,
             "vs_exact": vs_exact,
         }
+        if diag is not None:
+            line["diagnostics"] = diag
         print(json.dumps(line), flush=True)
     ha.close()
     if world > 1:
@@ -427,6 +444,8 @@ def main():
                     help="run the workload with this many heads instead of its own (small profiler captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-exact", action="store_true", help="skip the same-box exact-attention comparison")
+    ap.add_argument("--diagnostics", action="store_true",
+                    help="also report the hardness diagnostics (alpha, kappa) of the first 4096 rows of head 0")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

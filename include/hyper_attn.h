@@ -119,6 +119,26 @@ HA_API int hyper_attn_exact(hyper_attn_t h, const void *Q, const void *K, const 
                             int64_t n, int d, int heads, int causal);
 
 /*
+ * Hardness diagnostics of the attention matrices of small non-causal problems ("HyperAttention: Long-context
+ * Attention in Near-Linear Time", research-map summary, "Approach" and "Key results", abstract page: the
+ * guarantee rests on the max column norm of the normalised attention matrix and on the ratio of row norms
+ * once the large entries are removed). For each (batch, head) problem b, with A_ij = exp(q_i . k_j) and
+ * W = D^-1 A (the softmax matrix):
+ *   alpha[b] = n * max_{j >= first_col} sum_i W_ij^2   (1 for uniform attention; first_col > 0 leaves out
+ *              the first columns, e.g. sink-like heavy columns);
+ *   kappa[b] = max_i R_i / min_i R_i, R_i = the sum of A_ij over the columns outside row i's block of the
+ *              sortLSH order that hyper_attn_forward would use for (block, r, seed) (NaN when no row has
+ *              such columns, +inf when only some rows have none).
+ * Q, K: device pointers as for hyper_attn_forward (the handle's dtype and batch). alpha, kappa: HOST arrays
+ * of batch*heads doubles. Every entry of A is visited, so n <= 16384. Synchronous: returns after the values
+ * are on the host. Errors: HA_ERR_INVALID_ARG for null pointers, n > 16384, first_col outside [0, n) or an
+ * invalid shape.
+ */
+HA_API int hyper_attn_diagnostics(hyper_attn_t h, const void *Q, const void *K, int64_t n, int d, int heads,
+                                  int block, int r, uint64_t seed, int64_t first_col, double *alpha,
+                                  double *kappa);
+
+/*
  * Same computation with HOST buffers: copies Q, K, V to handle-owned device buffers, runs the forward
  * pass, copies O back and waits. Returns when O is valid on the host. The (batch, head) problems go
  * through in up to 8 contiguous groups so that host-to-device copies, the forward pass (on the handle's

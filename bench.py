@@ -346,9 +346,10 @@ def run_ours(args, w: wl.Workload):
                     "note": "exact softmax attention on the same inputs and GPU; causal counts half the pairs"}
         del O2
 
-    # optional: hardness diagnostics on the first rows of head 0 (every entry of A is visited, so a slice)
+    # optional: hardness diagnostics on the first rows of head 0 (every entry of A is visited, so a slice; the
+    # non-causal matrix of the slice, also for causal workloads)
     diag = None
-    if args.diagnostics and rank == 0 and not w.causal:
+    if args.diagnostics and rank == 0:
         nd = min(w.n, 4096)
         Qs, Ks = Q[:1, :nd].contiguous(), K[:1, :nd].contiguous()
         ha.set_options(dtype=w.dtype, batch=1, causal_base=w.base or 4096, stream=stream.cuda_stream, kernel=args.kernel)

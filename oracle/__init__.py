@@ -60,6 +60,11 @@ def _load():
                                 ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_uint64, ctypes.c_int64,
                                 vp, ctypes.c_int64, _f64p, vp, vp, vp, vp, vp]
     lib.ora_forward.restype = ctypes.c_int
+    lib.ora_forward_sampling.argtypes = lib.ora_forward.argtypes + [ctypes.c_int]
+    lib.ora_forward_sampling.restype = ctypes.c_int
+    lib.ora_draw_rownorm.argtypes = [ctypes.c_uint64, ctypes.c_int64, ctypes.c_int64, _f32p, ctypes.c_int64,
+                                     ctypes.c_int, ctypes.c_int, _i32p, _f64p]
+    lib.ora_draw_rownorm.restype = ctypes.c_int
     lib.ora_level_perms.argtypes = [_u16p, ctypes.c_int64, ctypes.c_int, _i32p, _i32p]
     lib.ora_level_perms.restype = ctypes.c_int
     lib.ora_exact_attention.argtypes = [_f32p, _f32p, _f32p, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
@@ -107,6 +112,20 @@ def draw_samples(seed: int, bh: int, node: int, N: int, m: int) -> np.ndarray:
     return S[:m].copy()
 
 
+def draw_rownorm(seed: int, bh: int, node: int, V: np.ndarray, m: int):
+    """m row-norm draws over the rows of V (N, d) float32: indices (int32, -1 when every row is zero) and the
+    log weights log(1 / (m p_j)), p_j = ||v_j||^2 / sum ||v||^2 (see oracle.c)."""
+    V = np.ascontiguousarray(V, np.float32)
+    N, d = V.shape
+    S = np.zeros(max(m, 1), np.int32)
+    lw = np.zeros(max(m, 1), np.float64)
+    _check(_load().ora_draw_rownorm(seed, bh, node, V, N, d, m, S, lw), "draw_rownorm")
+    return S[:m].copy(), lw[:m].copy()
+
+
+SAMPLING = {"uniform": 0, "rownorm": 1}
+
+
 def gray_rank(h: int) -> int:
     return int(_load().ora_gray_rank(h))
 
@@ -141,10 +160,11 @@ def level_perms(rank: np.ndarray, n: int, level: int):
 
 
 def forward(Q, K, V, *, block: int, m: int, r: int, causal: bool, seed: int, bh: int = 0,
-            base: int = 0, rows=None, want_parts: bool = False):
+            base: int = 0, rows=None, want_parts: bool = False, sampling: str = "uniform"):
     """One (batch*head) problem. Q, K, V: (n, d) float32 (bf16 inputs passed as their exact float32
     values). Returns a dict with O (nrows, d) float64, L (log of the estimated normaliser), and when
-    requested L1/L2 (non-causal only), rank (2n,) and near (2n,)."""
+    requested L1/L2 (non-causal only), rank (2n,) and near (2n,). sampling "uniform" reuses the uniform
+    samples for the product with V; "rownorm" draws that product's samples by the squared row norms of V."""
     Q = np.ascontiguousarray(Q, np.float32)
     K = np.ascontiguousarray(K, np.float32)
     V = np.ascontiguousarray(V, np.float32)
@@ -157,8 +177,9 @@ def forward(Q, K, V, *, block: int, m: int, r: int, causal: bool, seed: int, bh:
     L2 = np.zeros(max(nsel, 1), np.float64) if (want_parts and not causal) else None
     rank = np.zeros(2 * n, np.uint16)
     near = np.zeros(2 * n, np.uint8)
-    rc = _load().ora_forward(Q, K, V, n, d, block, m, r, int(causal), base, seed, bh,
-                             _ptr(sel), nsel, O, _ptr(L), _ptr(L1), _ptr(L2), _ptr(rank), _ptr(near))
+    rc = _load().ora_forward_sampling(Q, K, V, n, d, block, m, r, int(causal), base, seed, bh,
+                                      _ptr(sel), nsel, O, _ptr(L), _ptr(L1), _ptr(L2), _ptr(rank), _ptr(near),
+                                      SAMPLING[sampling])
     _check(rc, "forward")
     out = {"O": O[:nsel], "L": L[:nsel], "rank": rank, "near": near}
     if L1 is not None:

@@ -262,6 +262,54 @@ static void merge_part(double *O, double *L, const double *Op, double Lp, int d)
 }
 
 /*
+ * Row-norm samples of one problem ("Approach": the product with values via row-norm sampling).
+ * READING: m draws, independent and with replacement, of a key row j with probability p_j = ||v_j||^2 /
+ * sum_j' ||v_j'||^2 over the problem's N value rows; draw t carries the weight 1/(m p_j), so that the sum of
+ * weight * a_j v_j over the draws is an unbiased estimate of sum_j a_j v_j. The squared norms are sequential
+ * fp32 fused multiply-adds over k = 0..d-1 from +0 (a decision taken in fp32, the same on both sides); draw t
+ * uses u_t = (w >> 11) * 2^-53 with w = output word t mod 4 of Philox4x64-10 under key (seed, 3) at counter
+ * (t / 4, node, bh, 0), and picks the smallest j whose cumulative sum (double, index order) exceeds u_t times
+ * the total. logw[t] = log(1 / (m p_j)). If every norm is zero, S[t] = -1 (no draw).
+ */
+int ora_draw_rownorm(uint64_t seed, int64_t bh, int64_t node, const float *Vk, int64_t N, int d, int m,
+                     int32_t *S, double *logw)
+{
+    if (N <= 0 || m < 0) return ORA_EINVAL;
+    if (m == 0) return ORA_OK;
+    double *cdf = (double *)malloc(sizeof(double) * (size_t)N);
+    float *nrm = (float *)malloc(sizeof(float) * (size_t)N);
+    if (!cdf || !nrm) { free(cdf); free(nrm); return ORA_ENOMEM; }
+    double run = 0.0;
+    for (int64_t j = 0; j < N; ++j) {
+        float a = 0.0f;
+        for (int k = 0; k < d; ++k) a = fmaf(Vk[j * d + k], Vk[j * d + k], a);
+        nrm[j] = a;
+        run += (double)a;
+        cdf[j] = run;
+    }
+    const double total = run;
+    uint64_t key[2] = {seed, 3}, out4[4] = {0, 0, 0, 0};
+    for (int t = 0; t < m; ++t) {
+        if ((t & 3) == 0) {
+            uint64_t ctr[4] = {(uint64_t)(t / 4), (uint64_t)node, (uint64_t)bh, 0};
+            ora_philox4x64_10(ctr, key, out4);
+        }
+        if (total <= 0.0) { S[t] = -1; logw[t] = -INFINITY; continue; }
+        const double u = (double)(out4[t & 3] >> 11) * 0x1.0p-53;
+        const double target = u * total;
+        int64_t lo = 0, hi = N - 1;            /* smallest j with cdf[j] > target */
+        while (lo < hi) {
+            int64_t mid = lo + (hi - lo) / 2;
+            if (cdf[mid] > target) hi = mid; else lo = mid + 1;
+        }
+        S[t] = (int32_t)lo;
+        logw[t] = log(total / ((double)m * (double)nrm[lo]));
+    }
+    free(cdf); free(nrm);
+    return ORA_OK;
+}
+
+/*
  * The non-causal HyperAttention problem on N queries and N keys ("Approach"):
  *   1. sort queries and keys by hash rank (rq, rk);
  *   2. sorted query block i = positions [i*b', (i+1)*b'), b' = min(block, N) (READING: aligned diagonal
@@ -277,6 +325,7 @@ static void merge_part(double *O, double *L, const double *Op, double Lp, int d)
  */
 static int hyper_subproblem(const float *Qr, const float *Kr, const float *Vr, int64_t N, int d,
                             const uint16_t *rq, const uint16_t *rk, int64_t block, const int32_t *S, int m,
+                            const int32_t *Srn, const double *lwrn,
                             const int64_t *qsel, int64_t nsel,
                             double *Oout, double *Lout, double *L1out, double *L2out)
 {
@@ -295,7 +344,7 @@ static int hyper_subproblem(const float *Qr, const float *Kr, const float *Vr, i
 
 #pragma omp parallel
     {
-        double *sc = (double *)malloc(sizeof(double) * (size_t)(bp + m + 1));
+        double *sc = (double *)malloc(sizeof(double) * (size_t)(bp + 2 * m + 1));
         double *n1 = (double *)malloc(sizeof(double) * (size_t)d);
         double *n2 = (double *)malloc(sizeof(double) * (size_t)d);
 #pragma omp for schedule(dynamic, 16)
@@ -315,6 +364,13 @@ static int hyper_subproblem(const float *Qr, const float *Kr, const float *Vr, i
                 sc[bp + u] = dot_fd(qv, Kr + s * d, d);
                 if (sc[bp + u] > mx) mx = sc[bp + u];
             }
+            /* row-norm variant: the numerator's sampled part comes from the row-norm draws */
+            for (int u = 0; Srn && u < m; ++u) {
+                int64_t s = Srn[u];
+                if (s < 0 || posK[s] / bp == i) { sc[bp + m + u] = -INFINITY; continue; }
+                sc[bp + m + u] = dot_fd(qv, Kr + s * d, d);
+                if (sc[bp + m + u] > mx) mx = sc[bp + m + u];
+            }
             double d1 = 0.0, d2 = 0.0;
             for (int k = 0; k < d; ++k) { n1[k] = 0.0; n2[k] = 0.0; }
             for (int64_t j = 0; j < bp; ++j) {
@@ -328,6 +384,13 @@ static int hyper_subproblem(const float *Qr, const float *Kr, const float *Vr, i
                 double e = wsamp * exp(sc[bp + u] - mx);
                 const float *v = Vr + (int64_t)S[u] * d;
                 d2 += e;
+                if (!Srn)
+                    for (int k = 0; k < d; ++k) n2[k] += e * (double)v[k];
+            }
+            for (int u = 0; Srn && u < m; ++u) {
+                if (sc[bp + m + u] == -INFINITY) continue;
+                double e = exp(sc[bp + m + u] - mx + lwrn[u]);
+                const float *v = Vr + (int64_t)Srn[u] * d;
                 for (int k = 0; k < d; ++k) n2[k] += e * (double)v[k];
             }
             double dt = d1 + d2;
@@ -385,11 +448,29 @@ static int valid_causal_shape(int64_t n, int64_t base)
  * For causal = 0 only: L1, L2 (may be NULL) per produced row, as in hyper_subproblem.
  * rank_out (may be NULL): 2n ranks (Q rows then K rows); near_out (may be NULL): 2n flags.
  */
+/* sampling 0: the product with V reuses the uniform samples; 1: it uses row-norm samples (ora_draw_rownorm). */
+int ora_forward_sampling(const float *Q, const float *K, const float *V, int64_t n, int d, int64_t block, int m,
+                         int r, int causal, int64_t base, uint64_t seed, int64_t bh,
+                         const int64_t *rows, int64_t nrows,
+                         double *O, double *L, double *L1, double *L2, uint16_t *rank_out, uint8_t *near_out,
+                         int sampling);
+
 int ora_forward(const float *Q, const float *K, const float *V, int64_t n, int d, int64_t block, int m, int r,
                 int causal, int64_t base, uint64_t seed, int64_t bh,
                 const int64_t *rows, int64_t nrows,
                 double *O, double *L, double *L1, double *L2, uint16_t *rank_out, uint8_t *near_out)
 {
+    return ora_forward_sampling(Q, K, V, n, d, block, m, r, causal, base, seed, bh, rows, nrows, O, L, L1, L2,
+                                rank_out, near_out, 0);
+}
+
+int ora_forward_sampling(const float *Q, const float *K, const float *V, int64_t n, int d, int64_t block, int m,
+                         int r, int causal, int64_t base, uint64_t seed, int64_t bh,
+                         const int64_t *rows, int64_t nrows,
+                         double *O, double *L, double *L1, double *L2, uint16_t *rank_out, uint8_t *near_out,
+                         int sampling)
+{
+    if (sampling != 0 && sampling != 1) return ORA_EINVAL;
     if (n <= 0 || d <= 0 || block <= 0 || m < 0 || r < 0 || r > 16) return ORA_EINVAL;
     if (causal && !valid_causal_shape(n, base)) return ORA_EINVAL;
     int64_t nsel = rows ? nrows : n;
@@ -412,12 +493,15 @@ int ora_forward(const float *Q, const float *K, const float *V, int64_t n, int d
     if (!causal) {
         if (m > n) { rc = ORA_EINVAL; goto out; }
         int32_t *S = (int32_t *)malloc(sizeof(int32_t) * (size_t)(m > 0 ? m : 1));
-        if (!S) { rc = ORA_ENOMEM; goto out; }
+        int32_t *Srn = (int32_t *)malloc(sizeof(int32_t) * (size_t)(m > 0 ? m : 1));
+        double *lw = (double *)malloc(sizeof(double) * (size_t)(m > 0 ? m : 1));
+        if (!S || !Srn || !lw) { free(S); free(Srn); free(lw); rc = ORA_ENOMEM; goto out; }
         rc = ora_draw_samples(seed, bh, 1, n, m, S);
+        if (rc == ORA_OK && sampling) rc = ora_draw_rownorm(seed, bh, 1, V, n, d, m, Srn, lw);
         if (rc == ORA_OK)
-            rc = hyper_subproblem(Q, K, V, n, d, rank, rank + n, block, S, m, sel, nsel,
-                                  O, L ? L : Lloc, L1, L2);
-        free(S);
+            rc = hyper_subproblem(Q, K, V, n, d, rank, rank + n, block, S, m, sampling ? Srn : NULL,
+                                  sampling ? lw : NULL, sel, nsel, O, L ? L : Lloc, L1, L2);
+        free(S); free(Srn); free(lw);
         goto out;
     }
 
@@ -454,21 +538,24 @@ int ora_forward(const float *Q, const float *K, const float *V, int64_t n, int d
                 double *Op = (double *)malloc(sizeof(double) * (size_t)(cnt * d));
                 double *Lp = (double *)malloc(sizeof(double) * (size_t)cnt);
                 int32_t *S = (int32_t *)malloc(sizeof(int32_t) * (size_t)(m > 0 ? m : 1));
-                if (!lq || !ts || !Op || !Lp || !S) rc = ORA_ENOMEM;
+                int32_t *Srn = (int32_t *)malloc(sizeof(int32_t) * (size_t)(m > 0 ? m : 1));
+                double *lw = (double *)malloc(sizeof(double) * (size_t)(m > 0 ? m : 1));
+                if (!lq || !ts || !Op || !Lp || !S || !Srn || !lw) rc = ORA_ENOMEM;
                 if (rc == ORA_OK && m > half) rc = ORA_EINVAL;
                 if (rc == ORA_OK) {
                     int64_t c = 0;
                     for (int64_t t = 0; t < nsel; ++t)
                         if (sel[t] >= s0 + half && sel[t] < s0 + len) { lq[c] = sel[t] - (s0 + half); ts[c] = t; ++c; }
                     rc = ora_draw_samples(seed, bh, node, half, m, S);
+                    if (rc == ORA_OK && sampling) rc = ora_draw_rownorm(seed, bh, node, V + s0 * d, half, d, m, Srn, lw);
                 }
                 if (rc == ORA_OK)
                     rc = hyper_subproblem(Q + (s0 + half) * d, K + s0 * d, V + s0 * d, half, d,
-                                          rank + s0 + half, rank + n + s0, block, S, m, lq, cnt,
-                                          Op, Lp, NULL, NULL);
+                                          rank + s0 + half, rank + n + s0, block, S, m, sampling ? Srn : NULL,
+                                          sampling ? lw : NULL, lq, cnt, Op, Lp, NULL, NULL);
                 if (rc == ORA_OK)
                     for (int64_t c = 0; c < cnt; ++c) merge_part(O + ts[c] * d, &Lloc[ts[c]], Op + c * d, Lp[c], d);
-                free(lq); free(ts); free(Op); free(Lp); free(S);
+                free(lq); free(ts); free(Op); free(Lp); free(S); free(Srn); free(lw);
             }
         }
     }

@@ -393,3 +393,149 @@ def test_diagnostics_alpha_ignores_row_order(ora):
     a0, _ = ora.diagnostics(Q, K, block=16, r=5, seed=2)
     a1, _ = ora.diagnostics(Q[rng.permutation(n)], K, block=16, r=5, seed=2)
     assert a1 == pytest.approx(a0, rel=1e-12)
+
+
+# ---------------------------------------------------------------- row-norm sampling of the product with V
+# "HyperAttention: Long-context Attention in Near-Linear Time" (summary page, "Approach"): the product of the
+# normalised attention with V may be approximated by sampling rows of V in proportion to their squared norms.
+
+def _philox_words(seed, bh, node, nblocks):
+    """Words of Philox4x64-10 under key (seed, 3) at counters (c, node, bh, 0), c = 0..nblocks-1 (numpy)."""
+    # numpy increments its 256-bit counter before each block: start one below (c=0, node, bh, 0)
+    start = [2**64 - 1, node - 1, bh, 0] if node > 0 else [2**64 - 1, 2**64 - 1, bh - 1, 0]
+    g = np.random.Philox(key=np.array([seed, 3], np.uint64), counter=np.array(start, np.uint64))
+    return g.random_raw(4 * nblocks).astype(np.uint64)
+
+
+def test_rownorm_draws_tiny_bruteforce(ora):
+    """Squared norms 1, 0, 3: p = (1/4, 0, 3/4); a draw is row 0 exactly when u < 1/4, else row 2, and its
+    weight is 1/(m p)."""
+    V = np.zeros((3, 4), np.float32)
+    V[0, 0] = 1.0
+    V[2, :3] = 1.0
+    m, seed, bh, node = 11, 77, 2, 5
+    S, lw = ora.draw_rownorm(seed, bh, node, V, m)
+    w = _philox_words(seed, bh, node, (m + 3) // 4)
+    u = (w[:m] >> np.uint64(11)).astype(np.float64) * 2.0**-53
+    expect = np.where(u < 0.25, 0, 2)
+    assert np.array_equal(S, expect)
+    p = np.array([0.25, 0.0, 0.75])
+    np.testing.assert_allclose(np.exp(lw), 1.0 / (m * p[expect]), rtol=1e-14)
+    assert 0 < (expect == 0).sum() < m
+
+
+def test_rownorm_draw_frequencies(ora):
+    rng = np.random.default_rng(31)
+    N, d, m = 60, 8, 200000
+    V = (rng.standard_normal((N, d)) * rng.uniform(0.1, 3.0, (N, 1))).astype(np.float32)
+    V[[4, 17, 59]] = 0.0
+    S, _ = ora.draw_rownorm(5, 1, 1, V, m)
+    cnt = np.bincount(S, minlength=N)
+    assert cnt[[4, 17, 59]].sum() == 0
+    p = (V.astype(np.float64) ** 2).sum(axis=1)
+    p /= p.sum()
+    keep = p > 0
+    chi2 = (((cnt[keep] - m * p[keep]) ** 2) / (m * p[keep])).sum()
+    assert stats.chi2.sf(chi2, keep.sum() - 1) > 1e-4
+    a = ora.draw_rownorm(5, 1, 1, V, 64)[0]
+    assert not np.array_equal(a, ora.draw_rownorm(5, 2, 1, V, 64)[0])
+    assert not np.array_equal(a, ora.draw_rownorm(5, 1, 2, V, 64)[0])
+    assert not np.array_equal(a, ora.draw_rownorm(6, 1, 1, V, 64)[0])
+
+
+def test_rownorm_all_zero_rows_draw_nothing(ora):
+    S, lw = ora.draw_rownorm(1, 0, 1, np.zeros((16, 8), np.float32), 5)
+    assert np.all(S == -1) and np.all(lw == -np.inf)
+    Q, K, _ = rand_qkv(128, 16, 3)
+    out = ora.forward(Q, K, np.zeros((128, 16), np.float32), block=16, m=8, r=3, causal=False, seed=1,
+                      sampling="rownorm")
+    assert np.all(out["O"] == 0.0)
+
+
+def _dense_rownorm_weights(n, rq, rk, block, S, lw):
+    """Numerator weights of one problem: 1 on same-block pairs, sum of exp(lw) over draws of column j outside
+    the query's block."""
+    W = weights_noncausal(rq, rk, n, block, np.zeros(0, np.int64))
+    bp = min(block, n)
+    pq = np.argsort(rq, kind="stable")
+    pk = np.argsort(rk, kind="stable")
+    blk_q = np.empty(n, np.int64); blk_q[pq] = np.arange(n) // bp
+    blk_k = np.empty(n, np.int64); blk_k[pk] = np.arange(n) // bp
+    add = np.zeros(n)
+    np.add.at(add, S[S >= 0], np.exp(lw[S >= 0]))
+    return W + np.where(blk_q[:, None] != blk_k[None, :], add[None, :], 0.0)
+
+
+@pytest.mark.parametrize("seed", [41, 42])
+@pytest.mark.parametrize("causal", [False, True])
+def test_rownorm_dense_bruteforce(ora, seed, causal):
+    """The whole estimate restated densely: numerator weights from the row-norm draws, normaliser weights
+    from the uniform draws (the same dense form as test_dense_bruteforce)."""
+    n, d, block, m, r, base, bh = 256, 16, 16, 12, 4, 32, 1
+    Q, K, V = rand_qkv(n, d, seed)
+    P = ora.draw_projection(seed, d, r)
+    rq_all, aq = ranks_np(Q, P)
+    rk_all, ak = ranks_np(K, P)
+    X = np.concatenate([Q, K]).astype(np.float64)
+    assert (np.concatenate([aq, ak]) >= 1e-5 * np.linalg.norm(X, axis=1)[:, None]).all()
+    if causal:
+        Wd, _ = _dense_causal_weights(Q, K, P, block, base, m, seed, bh, ora)
+        Wn = np.zeros((n, n))
+        for q in range(n):
+            lo = q - q % base
+            Wn[q, lo:q + 1] = 1.0
+
+        def rec(node, s, length):
+            if length <= base:
+                return
+            h = length // 2
+            rec(2 * node, s, h)
+            rec(2 * node + 1, s + h, h)
+            S, lw = ora.draw_rownorm(seed, bh, node, V[s:s + h], m)
+            Wn[s + h:s + length, s:s + h] = _dense_rownorm_weights(h, rq_all[s + h:s + length], rk_all[s:s + h],
+                                                                   block, S, lw)
+        rec(1, 0, n)
+    else:
+        Wd = weights_noncausal(rq_all, rk_all, n, block, ora.draw_samples(seed, bh, 1, n, m))
+        S, lw = ora.draw_rownorm(seed, bh, 1, V, m)
+        Wn = _dense_rownorm_weights(n, rq_all, rk_all, block, S, lw)
+    Sc = Q.astype(np.float64) @ K.astype(np.float64).T
+    mx = np.where(Wd > 0, Sc, -np.inf).max(axis=1, keepdims=True)
+    E = np.exp(Sc - mx)
+    ref = ((Wn * E) @ V.astype(np.float64)) / (Wd * E).sum(axis=1, keepdims=True)
+    out = ora.forward(Q, K, V, block=block, m=m, r=r, causal=causal, base=base, seed=seed, bh=bh, sampling="rownorm")
+    np.testing.assert_allclose(out["O"], ref, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(out["L"], mx[:, 0] + np.log((Wd * E).sum(axis=1)), rtol=0, atol=1e-10)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_rownorm_single_value_row_is_exact(ora, causal):
+    """With one nonzero value row every draw picks it with weight 1/m, so the estimated numerator (output times
+    estimated normaliser) is exactly the numerator of exact attention."""
+    n, d = 256, 16
+    Q, K, V = rand_qkv(n, d, 9)
+    j0 = 70
+    V1 = np.zeros_like(V)
+    V1[j0] = V[j0]
+    Sc = Q.astype(np.float64) @ K.astype(np.float64).T
+    if causal:
+        Sc = np.where(np.tril(np.ones((n, n), bool)), Sc, -np.inf)
+    num = np.exp(Sc[:, j0])[:, None] * V1[j0].astype(np.float64)[None, :]
+    for seed in (1, 2, 3):
+        out = ora.forward(Q, K, V1, block=16, m=10, r=4, causal=causal, base=32, seed=seed, sampling="rownorm")
+        np.testing.assert_allclose(out["O"] * np.exp(out["L"])[:, None], num, rtol=1e-10, atol=1e-300)
+
+
+def test_rownorm_numerator_unbiased(ora):
+    """Over independent draws the mean estimated numerator (output times estimated normaliser) is the exact
+    numerator A V: within 5 standard errors per entry."""
+    n, d, block, m, r, T = 64, 8, 8, 8, 3, 4000
+    Q, K, V = rand_qkv(n, d, 16, planted=0.2)
+    ref = np.exp(Q.astype(np.float64) @ K.astype(np.float64).T) @ V.astype(np.float64)
+    est = np.zeros((T, n, d))
+    for seed in range(T):
+        out = ora.forward(Q, K, V, block=block, m=m, r=r, causal=False, seed=seed, sampling="rownorm")
+        est[seed] = out["O"] * np.exp(out["L"])[:, None]
+    se = est.std(axis=0, ddof=1) / np.sqrt(T)
+    z = (est.mean(axis=0) - ref) / se
+    assert np.abs(z).max() < 5.0, np.abs(z).max()

@@ -16,7 +16,8 @@ LIB_PATH = os.path.join(_HERE, "libhyper_attn.so")
 HA_OK, HA_ERR_INVALID_ARG, HA_ERR_UNSUPPORTED, HA_ERR_CUDA, HA_ERR_OOM, HA_ERR_TIMEOUT = 0, -1, -2, -3, -4, -5
 DTYPES = {"bf16": 0, "fp32": 1}
 KERNELS = {"auto": 0, "simt": 1, "tc": 2}
-DBG = {"rank": 0, "near": 1, "perm": 2, "inv": 3, "lse": 4}
+DBG = {"rank": 0, "near": 1, "perm": 2, "inv": 3, "lse": 4, "rn_s": 5, "rn_logw": 6}
+SAMPLING = {"uniform": 0, "rownorm": 1}
 
 # every symbol include/hyper_attn.h declares
 EXPORTS = [
@@ -27,7 +28,7 @@ EXPORTS = [
     "hyper_attn_last_kernel", "hyper_attn_forward_noalloc", "hyper_attn_exact",
     "hyper_attn_diagnostics",
 ]
-KERNEL_CLASSES = ["hash", "sort", "attn", "causal_base"]
+KERNEL_CLASSES = ["hash", "sort", "attn", "causal_base", "draws"]
 
 
 class HAError(RuntimeError):
@@ -47,6 +48,7 @@ class Options(ctypes.Structure):
         ("debug_captures", ctypes.c_int),
         ("bh_offset", ctypes.c_int64),
         ("test_stall_ms", ctypes.c_int),
+        ("sampling", ctypes.c_int),
     ]
 
 
@@ -140,7 +142,7 @@ class HyperAttention:
             raise HAError(rc, lib().hyper_attn_last_error(self._h).decode())
 
     def set_options(self, *, dtype="bf16", out_dtype=None, batch=1, causal_base=4096, stream=None,
-                    kernel="auto", debug_captures=False, bh_offset=0, test_stall_ms=0):
+                    kernel="auto", debug_captures=False, bh_offset=0, test_stall_ms=0, sampling="uniform"):
         o = Options()
         o.dtype = DTYPES[dtype]
         o.out_dtype = -1 if out_dtype is None else DTYPES[out_dtype]
@@ -151,6 +153,7 @@ class HyperAttention:
         o.debug_captures = int(bool(debug_captures))
         o.bh_offset = bh_offset
         o.test_stall_ms = test_stall_ms
+        o.sampling = SAMPLING[sampling]
         self._check(lib().hyper_attn_set_options(self._h, ctypes.byref(o)))
         self.options = o
 

@@ -37,6 +37,8 @@ struct hyper_attn_s {
         std::vector<size_t> perm, inv;
         std::vector<size_t> perm_bytes;
         size_t rank_bytes, near_bytes, lse_bytes;
+        // row-norm sampling (0 bytes when off): squared norms, chunk sums, cumulative sums, draws, log weights
+        size_t rn_nrm, rn_csum, rn_cdf, rn_S, rn_lw, rn_bytes;
     } lay{};
     bool have_last = false;
     int last_launches = 0;
@@ -180,7 +182,7 @@ void sort_passes(int r, ha::SortPass *p, int *np) {
 }
 
 // Lay out the workspace for shape s; returns total bytes.
-size_t plan_layout(const Shape &s, int esz_in, int capture, hyper_attn_s::Layout *L) {
+size_t plan_layout(const Shape &s, int esz_in, int capture, bool rownorm, hyper_attn_s::Layout *L) {
     size_t off = 0;
     auto take = [&](size_t bytes) { size_t o = off; off += align_up(bytes ? bytes : 1); return o; };
     L->status = take(256);
@@ -210,6 +212,14 @@ size_t plan_layout(const Shape &s, int esz_in, int capture, hyper_attn_s::Layout
     const size_t half_rows = static_cast<size_t>(s.bh) * (s.n / 2);
     L->Opart = take(s.causal ? sizeof(float) * s.levels * half_rows * s.d : 0);
     L->Lpart = take(s.causal ? sizeof(float) * s.levels * half_rows : 0);
+    const ha::RowNormGeom g = ha::rownorm_geometry(s.n, s.causal, s.levels, s.m, s.nodes_total);
+    const size_t draws = rownorm ? static_cast<size_t>(s.bh) * s.nodes_total * s.m : 0;
+    L->rn_nrm = take(rownorm ? sizeof(float) * s.bh * s.n : 0);
+    L->rn_csum = take(rownorm ? sizeof(double) * s.bh * g.slots : 0);
+    L->rn_cdf = take(rownorm ? sizeof(double) * s.bh * g.per_prob : 0);
+    L->rn_bytes = draws * 4;
+    L->rn_S = take(L->rn_bytes);
+    L->rn_lw = take(L->rn_bytes);
     L->end = off;
     (void)esz_in;
     return off;
@@ -314,8 +324,9 @@ int run_forward(hyper_attn_t h, const void *Q, const void *K, const void *V, voi
         use_tc = dtype == HA_DTYPE_BF16;
     }
 
+    const bool rownorm = h->opt.sampling == HA_SAMPLING_ROWNORM && s.m > 0 && !sort_only;
     hyper_attn_s::Layout lay;
-    const size_t bytes = plan_layout(s, esz, h->opt.debug_captures, &lay);
+    const size_t bytes = plan_layout(s, esz, h->opt.debug_captures, rownorm, &lay);
     int rc = ensure_workspace(h, bytes);
     if (rc) return rc;
     // a layout change invalidates resident draws only if their offsets moved
@@ -369,8 +380,26 @@ int run_forward(hyper_attn_t h, const void *Q, const void *K, const void *V, voi
         return HA_OK;
     };
 
-    long ev = prof_begin();
-    int kl = ha::launch_hash(Q, K, dtype, s.bh, s.n, s.d, P, s.r, rank, near, st);
+    const int32_t *Srn = nullptr;
+    const float *lwrn = nullptr;
+    long ev;
+    int kl;
+    if (rownorm) {
+        const ha::RowNormGeom g = ha::rownorm_geometry(s.n, s.causal, s.levels, s.m, s.nodes_total);
+        int32_t *rS = reinterpret_cast<int32_t *>(ws + lay.rn_S);
+        float *rlw = reinterpret_cast<float *>(ws + lay.rn_lw);
+        ev = prof_begin();
+        kl = ha::launch_rownorm_draws(g, V, dtype, s.d, s.bh, seed, bh_offset, reinterpret_cast<float *>(ws + lay.rn_nrm),
+                                      reinterpret_cast<double *>(ws + lay.rn_csum),
+                                      reinterpret_cast<double *>(ws + lay.rn_cdf), rS, rlw, st);
+        prof_end(ev, HA_KC_DRAWS, kl);
+        if (kl == -2) return fail(h, HA_ERR_UNSUPPORTED, "row-norm sampling supports at most 65535 problems per call");
+        if ((rc = count(kl, "row-norm draws"))) return rc;
+        Srn = rS;
+        lwrn = rlw;
+    }
+    ev = prof_begin();
+    kl = ha::launch_hash(Q, K, dtype, s.bh, s.n, s.d, P, s.r, rank, near, st);
     prof_end(ev, HA_KC_HASH, kl);
     if ((rc = count(kl, "hash"))) return rc;
 
@@ -401,12 +430,13 @@ int run_forward(hyper_attn_t h, const void *Q, const void *K, const void *V, voi
         int k = -2;
         ev = prof_begin();
         if (use_tc) family = HA_KERNEL_TC;
-        if (use_tc) k = ha::launch_attn_tc(lv, Q, K, V, s.d, perm, inv, S, s.m, s.nodes_total, O, out_dtype, lse, Op,
-                                           Lp, status, st, stall_ns);
+        if (use_tc)
+            k = ha::launch_attn_tc(lv, Q, K, V, s.d, perm, inv, S, s.m, s.nodes_total, O, out_dtype, lse, Op, Lp,
+                                   status, st, stall_ns, Srn, lwrn);
         if (k == -2 && h->opt.kernel != HA_KERNEL_TC) family = HA_KERNEL_SIMT;
         if (k == -2 && h->opt.kernel != HA_KERNEL_TC)
             k = ha::launch_attn_simt(lv, Q, K, V, dtype, s.d, perm, inv, S, s.m, s.nodes_total, O, out_dtype, lse, Op,
-                                     Lp, st);
+                                     Lp, st, Srn, lwrn);
         prof_end(ev, HA_KC_ATTN, k);
         if ((rc = count(k, "attention"))) return rc;
     }
@@ -439,6 +469,8 @@ int validate_options(hyper_attn_t h, const ha_options *o) {
     if (o->bh_offset < 0 || o->bh_offset > (int64_t(1) << 40))
         return fail(h, HA_ERR_INVALID_ARG, "bh_offset out of range");
     if (o->test_stall_ms < 0 || o->test_stall_ms > 1000) return fail(h, HA_ERR_INVALID_ARG, "test_stall_ms out of range");
+    if (o->sampling != HA_SAMPLING_UNIFORM && o->sampling != HA_SAMPLING_ROWNORM)
+        return fail(h, HA_ERR_INVALID_ARG, "bad sampling");
     return HA_OK;
 }
 
@@ -465,6 +497,7 @@ void hyper_attn_default_options(ha_options *o) {
     o->debug_captures = 0;
     o->bh_offset = 0;
     o->test_stall_ms = 0;
+    o->sampling = HA_SAMPLING_UNIFORM;
 }
 
 int hyper_attn_version(void) { return kVersion; }
@@ -537,7 +570,7 @@ int hyper_attn_diagnostics(hyper_attn_t h, const void *Q, const void *K, int64_t
     cudaStream_t st = static_cast<cudaStream_t>(h->opt.stream);
     const int esz = h->opt.dtype == HA_DTYPE_BF16 ? 2 : 4;
     hyper_attn_s::Layout lay;
-    const size_t fwd_bytes = align_up(plan_layout(s, esz, h->opt.debug_captures, &lay));
+    const size_t fwd_bytes = align_up(plan_layout(s, esz, h->opt.debug_captures, false, &lay));
     const size_t diag_scratch = align_up(sizeof(float) * 4 * static_cast<size_t>(s.bh) * n);
     const size_t diag_out = sizeof(double) * 2 * static_cast<size_t>(s.bh);
     rc = ensure_workspace(h, fwd_bytes + diag_scratch + diag_out);   // the forward below reuses it as is
@@ -703,6 +736,8 @@ int hyper_attn_debug_copy(hyper_attn_t h, int what, int level, void *dst, size_t
         case HA_DBG_RANK: off = L.rank; avail = L.rank_bytes; break;
         case HA_DBG_NEAR: off = L.near; avail = L.near_bytes; break;
         case HA_DBG_LSE: off = L.lse; avail = L.lse_bytes; break;
+        case HA_DBG_RN_S: off = L.rn_S; avail = L.rn_bytes; break;
+        case HA_DBG_RN_LOGW: off = L.rn_lw; avail = L.rn_bytes; break;
         case HA_DBG_PERM:
         case HA_DBG_INV: {
             const int idx = h->dk_causal ? level - 1 : level;

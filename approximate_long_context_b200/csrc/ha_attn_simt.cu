@@ -10,6 +10,9 @@
 // One online softmax runs over both sets with the weight folded into the score as + log(N/m), which gives
 // O = (N1 + N2) / (D1 + D2) and the log normaliser L = log(D1 + D2). The gather of the permuted rows is
 // done here: rows are read through the permutation, no permuted copy is stored.
+// With row-norm sampling of the product with V ("Approach": rows of V drawn in proportion to their squared
+// norms), the uniform samples feed only the normaliser D2 and the row-norm draws, each with its own log
+// weight log(1 / (m p_j)), feed only the numerator N2; both share the running maximum.
 //
 // causal_base_simt_kernel: exact causal attention (key index <= query index) inside leaves of `leaf` rows,
 // then the log-space merge with the off-diagonal parts of every causal level the row belongs to (the
@@ -33,19 +36,22 @@ struct RowState {
 #pragma unroll
         for (int c = 0; c < DPL; ++c) o[c] = 0.0f;
     }
-    // add one key with score s (already including any log-weight) and value slice v
+    // add one key with score s (already including any log-weight) and value slice v, to the normaliser
+    // (TO_L) and/or to the numerator (TO_O)
+    template <bool TO_L = true, bool TO_O = true>
     __device__ void add(float s, const float (&v)[DPL]) {
         if (s > mx) {
             const float corr = expf(mx - s);   // 0 when mx = -inf
-            l = l * corr + 1.0f;
+            l = l * corr + (TO_L ? 1.0f : 0.0f);
 #pragma unroll
-            for (int c = 0; c < DPL; ++c) o[c] = o[c] * corr + v[c];
+            for (int c = 0; c < DPL; ++c) o[c] = o[c] * corr + (TO_O ? v[c] : 0.0f);
             mx = s;
         } else {
             const float e = expf(s - mx);
-            l += e;
+            if (TO_L) l += e;
 #pragma unroll
-            for (int c = 0; c < DPL; ++c) o[c] += e * v[c];
+            for (int c = 0; c < DPL; ++c)
+                if (TO_O) o[c] += e * v[c];
         }
     }
 };
@@ -61,7 +67,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) attn_simt_kernel(
     Level lv, const void *__restrict__ Q, const void *__restrict__ K, const void *__restrict__ V, int dtype,
     const int32_t *__restrict__ perm, const int32_t *__restrict__ inv, const int32_t *__restrict__ S, int m,
     int64_t nodes_total, void *__restrict__ O, int out_dtype, float *__restrict__ lse, float *__restrict__ Opart,
-    float *__restrict__ Lpart) {
+    float *__restrict__ Lpart, const int32_t *__restrict__ Srn, const float *__restrict__ lwrn) {
     constexpr int DPL = D / 32;
     const int lane = threadIdx.x & 31;
     const int64_t wg = static_cast<int64_t>(blockIdx.x) * kWarpsPerCta + (threadIdx.x >> 5);
@@ -104,8 +110,27 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) attn_simt_kernel(
 #pragma unroll
             for (int c = 0; c < DPL; ++c) part += q[c] * x[c];
             const float s = warp_sum(part) + logw;
+            if (Srn) {
+                st.add<true, false>(s, x);            // normaliser only
+            } else {
+                load_slice<DPL>(V, head + krow * D + col, dtype, x);
+                st.add(s, x);
+            }
+        }
+    }
+    if (Srn && m > 0) {
+        const int64_t set = (bhi * nodes_total + (lv.heap0 + node - 1)) * m;
+        for (int u = 0; u < m; ++u) {
+            const int32_t kl = Srn[set + u];
+            if (kl < 0 || invK[kl] / lv.bp == i) continue;
+            const int64_t krow = node_start + kl;
+            load_slice<DPL>(K, head + krow * D + col, dtype, x);
+            float part = 0.0f;
+#pragma unroll
+            for (int c = 0; c < DPL; ++c) part += q[c] * x[c];
+            const float s = warp_sum(part) + lwrn[set + u];
             load_slice<DPL>(V, head + krow * D + col, dtype, x);
-            st.add(s, x);
+            st.add<false, true>(s, x);                // numerator only
         }
     }
     const float inv_l = 1.0f / st.l;
@@ -177,15 +202,16 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) causal_base_simt_kernel(
 
 int launch_attn_simt(const Level &lv, const void *Q, const void *K, const void *V, int dtype, int d,
                      const int32_t *perm, const int32_t *inv, const int32_t *S, int m, int64_t nodes_total,
-                     void *O, int out_dtype, float *lse, float *Opart, float *Lpart, cudaStream_t st) {
+                     void *O, int out_dtype, float *lse, float *Opart, float *Lpart, cudaStream_t st,
+                     const int32_t *Srn, const float *lwrn) {
     const int64_t warps = lv.bh * lv.nodes * lv.seg_len;
     const int64_t grid = (warps + kWarpsPerCta - 1) / kWarpsPerCta;
     if (d == 64)
         attn_simt_kernel<64><<<static_cast<unsigned>(grid), kWarpsPerCta * 32, 0, st>>>(
-            lv, Q, K, V, dtype, perm, inv, S, m, nodes_total, O, out_dtype, lse, Opart, Lpart);
+            lv, Q, K, V, dtype, perm, inv, S, m, nodes_total, O, out_dtype, lse, Opart, Lpart, Srn, lwrn);
     else if (d == 128)
         attn_simt_kernel<128><<<static_cast<unsigned>(grid), kWarpsPerCta * 32, 0, st>>>(
-            lv, Q, K, V, dtype, perm, inv, S, m, nodes_total, O, out_dtype, lse, Opart, Lpart);
+            lv, Q, K, V, dtype, perm, inv, S, m, nodes_total, O, out_dtype, lse, Opart, Lpart, Srn, lwrn);
     else
         return -1;
     return cudaPeekAtLastError() == cudaSuccess ? 1 : -1;

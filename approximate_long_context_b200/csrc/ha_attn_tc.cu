@@ -13,6 +13,12 @@
 //  softmax over both parts gives O = (N1+N2)/(D1+D2); the epilogue writes each row to its original position
 //  (the merge and un-permute), or, for causal levels, the fp32 part and its log normaliser.
 //
+//  LEVEL_RN: LEVEL with row-norm sampling of the product with V ("Approach": rows of V drawn with probability
+//  proportional to their squared norms, weight 1/(m p_j)). The key stream gains ceil(m/128) chunks of the
+//  row-norm draws outside block i, each column with its own log2 weight; the uniform sample chunks feed only
+//  the normaliser (their P.V products are not issued and their V rows not loaded) and the row-norm chunks
+//  only the numerator, so O = (N1 + N2') / (D1 + D2).
+//
 //  CAUSAL: exact causal attention inside leaves of c rows (the summary's recursive causal extension: the
 //  base case), merged in log space with the parts of every causal level the row belongs to
 //  ("Limitations": partitioning and merging). A work item is a pair of query tiles of one leaf; query tile
@@ -56,6 +62,7 @@ constexpr int kThreads = 384;
 constexpr int kKC = 128;                // keys per chunk
 constexpr int kMaxLevels = 16;
 constexpr int kMaxSampleList = 1024;    // sampled columns per problem handled by the tensor-core path
+constexpr int kMaxSampleListRn = 256;   // the same with row-norm sampling (m uniform samples + m draws)
 constexpr int kMaxBlock = 1024;         // rows per sorted block handled by the tensor-core path
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -63,7 +70,8 @@ constexpr float kRescaleLog2 = 8.0f;   // rescale O only when the running max gr
 
 // MODE_DENSE: exact (non-causal) softmax attention of every query tile against every key chunk of its
 // sequence, with the CAUSAL mode's work layout (a "leaf" is the whole sequence) and no mask.
-enum { MODE_LEVEL = 0, MODE_CAUSAL = 1, MODE_DENSE = 2 };
+enum { MODE_LEVEL = 0, MODE_CAUSAL = 1, MODE_DENSE = 2, MODE_LEVEL_RN = 3 };
+__host__ __device__ constexpr bool is_level(int mode) { return mode == MODE_LEVEL || mode == MODE_LEVEL_RN; }
 
 struct TcArgs {
     int mode;
@@ -75,6 +83,9 @@ struct TcArgs {
     int m;
     int64_t nodes_total;
     int nb, ns;            // block chunks, sample chunks
+    const int32_t *Srn;    // LEVEL_RN: row-norm draws [bh][nodes_total][m] (local key row, -1: none)
+    const float *lwrn;     // LEVEL_RN: their natural-log weights log(1 / (m p_j))
+    int nr;                // LEVEL_RN: row-norm chunks (0 otherwise)
     int tiles_per_block, pairs_per_block;
     float lw2;             // log2(N / m)
     // CAUSAL
@@ -109,7 +120,7 @@ template <int MODE>
 __device__ __forceinline__ Item decode(const TcArgs &a, int64_t it64) {
     Item x{};
     const uint32_t it = static_cast<uint32_t>(it64);
-    if (MODE == MODE_LEVEL) {
+    if (is_level(MODE)) {
         const uint32_t prob = it / a.per_outer;
         const uint32_t rem = it - prob * a.per_outer;
         const uint32_t ppb = static_cast<uint32_t>(a.pairs_per_block);
@@ -123,8 +134,8 @@ __device__ __forceinline__ Item decode(const TcArgs &a, int64_t it64) {
         x.node = prob - bhi * nodes;
         x.v0 = x.pair * 2 < a.tiles_per_block;
         x.v1 = x.pair * 2 + 1 < a.tiles_per_block;
-        x.nc0 = x.v0 ? a.nb + a.ns : 0;
-        x.nc1 = x.v1 ? a.nb + a.ns : 0;
+        x.nc0 = x.v0 ? a.nb + a.ns + a.nr : 0;
+        x.nc1 = x.v1 ? a.nb + a.ns + a.nr : 0;
     } else {
         const uint32_t po = it / a.per_outer;
         const int pair = a.pairs_per_leaf - 1 - static_cast<int>(po);   // heaviest first
@@ -197,6 +208,13 @@ struct Cfg {
     static constexpr int kKPerm = kCacheB + kMaxSampleList * 4;            // key rows of the item's block
     static constexpr int kQPerm = kKPerm + kMaxBlock * 4;                  // query rows of one tile
     static constexpr int kRows = kQPerm + 128 * 4;                         // global rows of each stage
+    // LEVEL_RN (m <= kMaxSampleListRn): the uniform samples take entries [0, m) of the list and the caches, the
+    // row-norm draws [m, 2m); the upper halves hold the draws' log2 weights per problem (cache), per item (list)
+    // and per stage column
+    static constexpr int kCacheW = kCacheS + (kMaxSampleList / 2) * 4;
+    static constexpr int kListW = kList + (kMaxSampleList / 2) * 4;
+    static constexpr int kStageW = kCacheB + (kMaxSampleList / 2) * 4;
+    static constexpr int kZeroW = kCacheW + kMaxSampleListRn * 4;         // 128 zero weights (block chunks)
     static constexpr int kWord = kRows + NST * 128 * 4;
     static constexpr int kStage = (kWord + NST * 4 + 64 + 15) / 16 * 16;   // 8 softmax warps x 32 rows x SEG
     static constexpr int kBars = kStage + (kStageInQ ? 0 : 8 * 32 * SEG);
@@ -213,6 +231,9 @@ struct Cfg {
     static_assert(kStage % 16 == 0, "16-byte stage pieces");
     static_assert(!kStageInQ || 4 * 32 * SEG <= kTileBytes, "a tile's four warps stage in its Q buffer");
     static_assert(kBytes + 1024 <= 232448, "shared memory budget");
+    static_assert(2 * kMaxSampleListRn <= kMaxSampleList / 2 && NST * 128 <= kMaxSampleList / 2 &&
+                      kMaxSampleListRn + 128 <= kMaxSampleList / 2,
+                  "row-norm entries fit in the lower halves, their weights in the upper halves");
     static_assert(kOCol + 2 * D <= 512, "TMEM budget");
 };
 
@@ -286,10 +307,11 @@ __device__ __forceinline__ uint32_t swz(int slab, int row, int j) {
     return static_cast<uint32_t>(slab * (128 * 128) + row * 128 + ((j ^ (row & 7)) << 4));
 }
 
-// MODE (MODE_LEVEL or MODE_CAUSAL) is a compile-time parameter: each instance holds only its own mode's loads,
+// MODE (MODE_LEVEL, MODE_LEVEL_RN, MODE_CAUSAL or MODE_DENSE) is a compile-time parameter: each instance holds
+// only its own mode's loads,
 // masks and epilogue, which keeps the instruction footprint of the concurrently running roles small (measured:
 // about 4% faster than one instance for both modes).
-template <int D, int MODE>
+template <int D, int MODE, bool HOOK>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
     using C = Cfg<D>;
     extern __shared__ unsigned char smem_raw[];
@@ -303,6 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+    if (MODE == MODE_LEVEL_RN && threadIdx.x < kKC) reinterpret_cast<float *>(sm + C::kZeroW)[threadIdx.x] = 0.0f;
     if (threadIdx.x == 32) {
         for (int i = 0; i < 2 * C::QB; ++i) {
             mbar_init(bar(C::bQFull + i), 32);     // the Q loader's lanes (copy completion)
@@ -343,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
     // LEVEL items all cost the same: each CTA takes a contiguous range, so consecutive items share a problem
     // and its cached samples. CAUSAL items are ordered heaviest first and dealt round-robin.
     int64_t first, last, stride;
-    if (MODE == MODE_LEVEL) {
+    if (is_level(MODE)) {
         const int64_t per = (a.items + gridDim.x - 1) / gridDim.x;
         first = static_cast<int64_t>(blockIdx.x) * per;
         last = min(a.items, first + per);
@@ -371,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
             return false;
         const uint32_t base = sbase + C::kQ + (t * C::QB + qb) * C::kTileBytes;
         int64_t qbase;
-        const bool through_perm = MODE == MODE_LEVEL;
+        const bool through_perm = is_level(MODE);
         if (through_perm) {
             // the tile's 128 query rows: one 16-byte load per lane, staged in shared memory
             const int32_t *pq = a.perm + (x.prob * 2) * a.lv.seg_len + x.blk * a.lv.bp + (x.pair * 2 + t) * 128;
@@ -412,6 +435,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
         int32_t *cache_b = reinterpret_cast<int32_t *>(sm + C::kCacheB);
         int32_t *kperm = reinterpret_cast<int32_t *>(sm + C::kKPerm);
         int32_t *stage_rows = reinterpret_cast<int32_t *>(sm + C::kRows);
+        float *cache_w = reinterpret_cast<float *>(sm + C::kCacheW);
+        float *list_w = reinterpret_cast<float *>(sm + C::kListW);
+        float *stage_w = reinterpret_cast<float *>(sm + C::kStageW);
         int64_t cached_prob = -1;
         uint32_t g = 0;
         bool ok = true;
@@ -424,9 +450,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
             }
             // key rows of block blk and the compacted sample list of this item: the sampled columns whose key
             // lies outside block blk, in sample order (from the per-problem cache of samples and their blocks)
-            int cnt = 0;
+            int cnt = 0, cnt_rn = 0;
             int64_t kbase = 0;
-            if (MODE == MODE_LEVEL) {
+            if (is_level(MODE)) {
                 kbase = x.bhi * a.n + x.node * a.lv.node_len;
                 const int32_t *pkg = a.perm + (x.prob * 2 + 1) * a.lv.seg_len + x.blk * a.lv.bp;
                 __syncwarp();
@@ -440,6 +466,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                         for (int u = lane; u < a.m; u += 32) cache_s[u] = Sp[u];
                         __syncwarp();
                         for (int u = lane; u < a.m; u += 32) cache_b[u] = ik[cache_s[u]] / a.lv.bp;
+                        if (MODE == MODE_LEVEL_RN) {
+                            // row-norm draws of this problem behind the uniform samples; -1 (no draw) never kept
+                            const int64_t so = (x.bhi * a.nodes_total + (a.lv.heap0 + x.node - 1)) * a.m;
+                            for (int u = lane; u < a.m; u += 32) {
+                                cache_s[a.m + u] = a.Srn[so + u];
+                                cache_w[u] = a.lwrn[so + u] * kLog2e;
+                            }
+                            __syncwarp();
+                            for (int u = lane; u < a.m; u += 32) {
+                                const int32_t sr = cache_s[a.m + u];
+                                cache_b[a.m + u] = sr < 0 ? -1 : ik[sr] / a.lv.bp;
+                            }
+                        }
                         cached_prob = x.prob;
                     }
                     __syncwarp();
@@ -450,6 +489,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                         if (keep) slist[cnt + __popc(bal & lt_mask)] = cache_s[u];
                         cnt += __popc(bal);
                     }
+                    if (MODE == MODE_LEVEL_RN) {
+                        for (int base = 0; base < a.m; base += 32) {
+                            const int u = base + lane;
+                            const bool keep = u < a.m && cache_s[a.m + u] >= 0 && cache_b[a.m + u] != x.blk;
+                            const unsigned bal = __ballot_sync(0xffffffffu, keep);
+                            if (keep) {
+                                const int at = cnt_rn + __popc(bal & lt_mask);
+                                slist[a.m + at] = cache_s[a.m + u];
+                                list_w[at] = cache_w[u];
+                            }
+                            cnt_rn += __popc(bal);
+                        }
+                    }
                 }
                 __syncwarp();
             }
@@ -458,15 +510,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                 const uint32_t round = g / C::NST;
                 if (round > 0 && !mbar_wait(bar(C::bKVEmpty + slot), (round - 1) & 1, abort_flag)) { ok = false; break; }
                 int valid_cols = kKC;
-                int kind;   // 0: block chunk (through the key permutation), 1: sample chunk, 2: contiguous
+                // 0: block chunk (through the key permutation), 1: sample chunk, 2: contiguous, 3: row-norm chunk
+                int kind;
                 int u0 = 0;
-                if (MODE == MODE_LEVEL) {
+                if (is_level(MODE)) {
                     if (c < a.nb) {
                         kind = 0;
-                    } else {
+                    } else if (c < a.nb + a.ns) {
                         kind = 1;
                         u0 = (c - a.nb) * kKC;
                         valid_cols = min(kKC, max(0, cnt - u0));
+                    } else {
+                        kind = 3;
+                        u0 = (c - a.nb - a.ns) * kKC;
+                        valid_cols = min(kKC, max(0, cnt_rn - u0));
+                        if (MODE == MODE_LEVEL_RN) {
+                            for (int row = lane; row < kKC; row += 32)
+                                stage_w[slot * kKC + row] = row + u0 < cnt_rn ? list_w[u0 + row] : 0.0f;
+                            __syncwarp();
+                        }
                     }
                 } else {
                     kind = 2;
@@ -476,12 +538,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                     mbar_arrive(bar(C::bWordFull + slot));
                 }
                 // the chunk's 128 global rows, published for the V loader
-                const int64_t cbase = (MODE == MODE_LEVEL) ? kbase : x.leaf_start + static_cast<int64_t>(c) * kKC;
+                const int64_t cbase = is_level(MODE) ? kbase : x.leaf_start + static_cast<int64_t>(c) * kKC;
                 int32_t *rows = stage_rows + slot * 128;
                 for (int row = lane; row < kKC; row += 32) {
                     int32_t loc;
                     if (kind == 0) loc = kperm[c * kKC + row];
                     else if (kind == 1) loc = row + u0 < cnt ? slist[u0 + row] : 0;
+                    else if (kind == 3) loc = row + u0 < cnt_rn ? slist[a.m + u0 + row] : 0;
                     else loc = row;
                     rows[row] = static_cast<int32_t>(cbase + loc);
                 }
@@ -510,6 +573,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
             for (int c = 0; c < x.nc_max; ++c, ++g) {
                 const int slot = static_cast<int>(g % C::NST);
                 if (!mbar_wait(bar(C::bRowsFull + slot), (g / C::NST) & 1, abort_flag)) { ok = false; break; }
+                if (MODE == MODE_LEVEL_RN && c >= a.nb && c < a.nb + a.ns) {
+                    // uniform samples feed only the normaliser: no P.V product reads this stage's V
+                    mbar_arrive(bar(C::bKVFull + slot));
+                    continue;
+                }
                 const int32_t *rows = stage_rows + slot * 128;
                 const uint32_t vb = sbase + C::kV + slot * C::kTileBytes;
 #pragma unroll 8
@@ -648,10 +716,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                     // V of chunk c arrived with K (one barrier per stage), which S of this pair waited for
                     const uint64_t dv = dv0 + static_cast<uint64_t>((slot * C::kTileBytes) >> 4);
                     const uint32_t od = tmem + C::kOCol + t * D;
+                    // LEVEL_RN: the uniform sample chunks have no P.V product (the commits below still arrive)
+                    const bool pv = MODE != MODE_LEVEL_RN || c < a.nb || c >= a.nb + a.ns;
+                    if (pv) {
 #pragma unroll
-                    for (int kk = 0; kk < kKC / 16; ++kk) {
-                        const uint32_t pa = C::kSepP ? tmem + C::kPCol + t * 64 + kk * 8 : tmem + buf * 128 + kk * 8;
-                        mma_ts(od, pa, dv + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv, (c > 0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < kKC / 16; ++kk) {
+                            const uint32_t pa =
+                                C::kSepP ? tmem + C::kPCol + t * 64 + kk * 8 : tmem + buf * 128 + kk * 8;
+                            mma_ts(od, pa, dv + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv,
+                                   (c > 0 || kk > 0) ? 1u : 0u);
+                        }
                     }
                     // the tile's n-th P.V arrives on barrier 2t + (n & 1), phase n >> 1 (with P apart, this also
                     // frees the tile's P buffer)
@@ -764,10 +838,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                     // V of chunk c arrived with K (one barrier per stage), which S of this pair waited for
                     const uint64_t dv = dv0 + static_cast<uint64_t>((slot * C::kTileBytes) >> 4);
                     const uint32_t od = tmem + C::kOCol + t * D;
+                    if (MODE != MODE_LEVEL_RN || c < a.nb || c >= a.nb + a.ns) {
 #pragma unroll
-                    for (int kk = 0; kk < kKC / 16; ++kk)
-                        mma_ts(od, tmem + buf * 128 + kk * 8, dv + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv,
-                               (c > 0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < kKC / 16; ++kk)
+                            mma_ts(od, tmem + buf * 128 + kk * 8, dv + static_cast<uint64_t>((kk * 2048) >> 4),
+                                   idesc_pv, (c > 0 || kk > 0) ? 1u : 0u);
+                    }
                     // the tile's barrier first, then the ring buffer's: a waiter that has seen the buffer free may
                     // rely on the tile's barrier having arrived
                     uint32_t &pvn = t == 0 ? pvn0 : pvn1;
@@ -798,6 +874,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
         uint32_t pvt = 0;                            // P.V products of this tile before the current item
         int qn = 0;                                  // items of this tile so far (its Q buffer is qn mod QB)
         bool ok = true;
+        // test hook (its own instance: the check alone, even outside the chunk loop, measured about 15% slower
+        // on the long workload): the first wait targets a barrier nothing completes; it runs out, sets the
+        // abort flag, and every role stops
+        if (HOOK && a.stall_ns > 0 && first < last &&
+            !mbar_wait(bar(C::bNever), 0, abort_flag, static_cast<uint64_t>(a.stall_ns)))
+            ok = false;
         for (int64_t it = first; it < last && ok; it += stride) {
             const Item x = decode<MODE>(a, it);
             const bool my_valid = t == 0 ? x.v0 : x.v1;
@@ -805,7 +887,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
             const int my_gt = t == 0 ? x.gt0 : x.gt1;
             if (!my_valid) { kp += x.npairs; g += x.nc_max; continue; }
             int64_t qloc = 0;
-            if (MODE == MODE_LEVEL) {
+            if (is_level(MODE)) {
                 const int64_t pos = x.blk * a.lv.bp + (x.pair * 2 + t) * 128 + r;
                 qloc = a.perm[(x.prob * 2) * a.lv.seg_len + pos];   // consumed by the epilogue
             }
@@ -814,22 +896,30 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                 const uint32_t k = kp + static_cast<uint32_t>(pair_index(x, t, c));
                 const int buf = static_cast<int>(k % C::R);
                 const uint32_t tS = trow + buf * 128;
-                if (a.stall_ns > 0 && it == first && c == 0 &&
-                    !mbar_wait(bar(C::bNever), 0, abort_flag, static_cast<uint64_t>(a.stall_ns))) {
-                    ok = false;   // test hook: this wait runs out, sets the abort flag, and every role stops
-                    break;
-                }
                 if (!mbar_wait(bar(C::bSFull + buf), (k / C::R) & 1, abort_flag)) { ok = false; break; }
                 // column bound: columns > bound are masked (bound >= 127: none)
                 int bound = kKC - 1;
                 float w2 = 0.0f;
-                if (MODE == MODE_LEVEL) {
+                // LEVEL_RN: uniform sample chunks add to the normaliser only (no P is written), row-norm chunks
+                // (per-column log2 weights) to the numerator only
+                bool to_l = true, to_o = true;
+                // LEVEL_RN: every chunk's scores get per-column log2 weights, wcol[col] + w2 (zero for block
+                // chunks, log2(N/m) for uniform sample chunks, the draws' weights for row-norm chunks), so that
+                // the softmax runs one code path for all chunk kinds
+                const float *wcol = reinterpret_cast<const float *>(sm + C::kZeroW);
+                if (is_level(MODE)) {
                     if (c >= a.nb) {
                         const uint32_t gc = g + c;
                         const int slot = static_cast<int>(gc % C::NST);
                         if (!mbar_wait(bar(C::bWordFull + slot), (gc / C::NST) & 1, abort_flag)) { ok = false; break; }
                         bound = words[slot] - 1;
-                        w2 = a.lw2;
+                        if (MODE != MODE_LEVEL_RN || c < a.nb + a.ns) {
+                            w2 = a.lw2;
+                            to_o = MODE != MODE_LEVEL_RN;
+                        } else {
+                            wcol = reinterpret_cast<const float *>(sm + C::kStageW) + slot * kKC;
+                            to_l = false;
+                        }
                     }
                 } else {
                     bound = MODE == MODE_DENSE ? kKC - 1 : my_gt * 128 + r - c * kKC;
@@ -851,6 +941,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                             if (h * 64 + 32 + e > bound) vb[e] = 0xff800000u;
                         }
                     }
+                    if (MODE == MODE_LEVEL_RN) {
+                        // weighted base-2 scores (a masked -inf stays -inf); smax then holds the weighted max
+                        const float4 *w4 = reinterpret_cast<const float4 *>(wcol + h * 64);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const float4 wa = w4[e], wb = w4[8 + e];
+                            va[4 * e] = __float_as_uint(fmaf(__uint_as_float(va[4 * e]), kLog2e, wa.x + w2));
+                            va[4 * e + 1] = __float_as_uint(fmaf(__uint_as_float(va[4 * e + 1]), kLog2e, wa.y + w2));
+                            va[4 * e + 2] = __float_as_uint(fmaf(__uint_as_float(va[4 * e + 2]), kLog2e, wa.z + w2));
+                            va[4 * e + 3] = __float_as_uint(fmaf(__uint_as_float(va[4 * e + 3]), kLog2e, wa.w + w2));
+                            vb[4 * e] = __float_as_uint(fmaf(__uint_as_float(vb[4 * e]), kLog2e, wb.x + w2));
+                            vb[4 * e + 1] = __float_as_uint(fmaf(__uint_as_float(vb[4 * e + 1]), kLog2e, wb.y + w2));
+                            vb[4 * e + 2] = __float_as_uint(fmaf(__uint_as_float(vb[4 * e + 2]), kLog2e, wb.z + w2));
+                            vb[4 * e + 3] = __float_as_uint(fmaf(__uint_as_float(vb[4 * e + 3]), kLog2e, wb.w + w2));
+                        }
+                    }
                     float mx0 = __uint_as_float(va[0]), mx1 = __uint_as_float(vb[0]);
 #pragma unroll
                     for (int e = 1; e < 32; ++e) {
@@ -859,7 +965,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                     }
                     smax = fmaxf(smax, fmaxf(mx0, mx1));
                 }
-                const float xmax = smax == -INFINITY ? -INFINITY : fmaf(smax, kLog2e, w2);
+                const float xmax = smax == -INFINITY ? -INFINITY
+                                   : MODE == MODE_LEVEL_RN ? smax
+                                                                                : fmaf(smax, kLog2e, w2);
                 const float m_new = xmax > m_run + kRescaleLog2 ? xmax : m_run;
                 const bool grow = m_new != m_run;
                 const float alpha = grow ? ex2_approx(m_run - m_new) : 1.0f;   // 0 when m_run = -inf
@@ -913,20 +1021,43 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                         }
                     }
                     uint32_t pk[32];
+                    if (MODE == MODE_LEVEL_RN) {
+                        // P = 2^(x log2 e + w_col + w2 - m_run)
+                        const float4 *w4 = reinterpret_cast<const float4 *>(wcol + h * 64);
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const float p0 = ex2_approx(fmaf(__uint_as_float(va[2 * e]), kLog2e, off));
-                        const float p1 = ex2_approx(fmaf(__uint_as_float(va[2 * e + 1]), kLog2e, off));
-                        const float p2 = ex2_approx(fmaf(__uint_as_float(vb[2 * e]), kLog2e, off));
-                        const float p3 = ex2_approx(fmaf(__uint_as_float(vb[2 * e + 1]), kLog2e, off));
-                        l0 += p0 + p1;
-                        l1 += p2 + p3;
-                        pk[e] = pack_bf16x2(p0, p1);
-                        pk[16 + e] = pack_bf16x2(p2, p3);
+                        for (int e = 0; e < 8; ++e) {
+                            const float4 wa = w4[e], wb = w4[8 + e];
+                            const float a0 = ex2_approx(fmaf(__uint_as_float(va[4 * e]), kLog2e, wa.x + off));
+                            const float a1 = ex2_approx(fmaf(__uint_as_float(va[4 * e + 1]), kLog2e, wa.y + off));
+                            const float a2 = ex2_approx(fmaf(__uint_as_float(va[4 * e + 2]), kLog2e, wa.z + off));
+                            const float a3 = ex2_approx(fmaf(__uint_as_float(va[4 * e + 3]), kLog2e, wa.w + off));
+                            const float b0 = ex2_approx(fmaf(__uint_as_float(vb[4 * e]), kLog2e, wb.x + off));
+                            const float b1 = ex2_approx(fmaf(__uint_as_float(vb[4 * e + 1]), kLog2e, wb.y + off));
+                            const float b2 = ex2_approx(fmaf(__uint_as_float(vb[4 * e + 2]), kLog2e, wb.z + off));
+                            const float b3 = ex2_approx(fmaf(__uint_as_float(vb[4 * e + 3]), kLog2e, wb.w + off));
+                            l0 += (a0 + a1) + (a2 + a3);
+                            l1 += (b0 + b1) + (b2 + b3);
+                            pk[2 * e] = pack_bf16x2(a0, a1);
+                            pk[2 * e + 1] = pack_bf16x2(a2, a3);
+                            pk[16 + 2 * e] = pack_bf16x2(b0, b1);
+                            pk[16 + 2 * e + 1] = pack_bf16x2(b2, b3);
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const float p0 = ex2_approx(fmaf(__uint_as_float(va[2 * e]), kLog2e, off));
+                            const float p1 = ex2_approx(fmaf(__uint_as_float(va[2 * e + 1]), kLog2e, off));
+                            const float p2 = ex2_approx(fmaf(__uint_as_float(vb[2 * e]), kLog2e, off));
+                            const float p3 = ex2_approx(fmaf(__uint_as_float(vb[2 * e + 1]), kLog2e, off));
+                            l0 += p0 + p1;
+                            l1 += p2 + p3;
+                            pk[e] = pack_bf16x2(p0, p1);
+                            pk[16 + e] = pack_bf16x2(p2, p3);
+                        }
                     }
-                    tmem_st32(tP + h * 32, pk);
+                    if (to_o) tmem_st32(tP + h * 32, pk);
                 }
-                l += l0 + l1;
+                if (to_l) l += l0 + l1;
                 tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(bar(C::kSepP ? C::bPFullT + t : C::bPFull + buf));
@@ -952,7 +1083,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                     for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(o[e]) * scale;
                 };
             };
-            if (MODE == MODE_LEVEL) {
+            if (is_level(MODE)) {
                 const int64_t N = a.lv.seg_len;
                 if (a.lv.level == 0) {
                     const int64_t orow = x.bhi * a.n + a.lv.q_off + x.node * a.lv.node_len + qloc;
@@ -1048,13 +1179,13 @@ int num_sms() {
     return sms;
 }
 
-template <int D, int MODE>
+template <int D, int MODE, bool HOOK = false>
 int launch_tc(const void *Q, const void *K, const void *V, TcArgs args, cudaStream_t st) {
     args.Q = static_cast<const uint16_t *>(Q);
     args.K = static_cast<const uint16_t *>(K);
     args.V = static_cast<const uint16_t *>(V);
     const size_t smem = Cfg<D>::kBytes + 1024;
-    auto kern = attn_tc_kernel<D, MODE>;
+    auto kern = attn_tc_kernel<D, MODE, HOOK>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
         return -1;
     const int64_t grid = args.items < num_sms() ? args.items : num_sms();
@@ -1066,6 +1197,16 @@ int launch_tc(const void *Q, const void *K, const void *V, TcArgs args, cudaStre
 int dispatch(int d, const void *Q, const void *K, const void *V, const TcArgs &args, cudaStream_t st) {
     const bool level = args.mode == MODE_LEVEL;
     const bool dense = args.mode == MODE_DENSE;
+    if (args.mode == MODE_LEVEL_RN) {
+        if (d == 64) return launch_tc<64, MODE_LEVEL_RN>(Q, K, V, args, st);
+        if (d == 128) return launch_tc<128, MODE_LEVEL_RN>(Q, K, V, args, st);
+        return -2;
+    }
+    if (level && args.stall_ns > 0) {   // the test hook's instance
+        if (d == 64) return launch_tc<64, MODE_LEVEL, true>(Q, K, V, args, st);
+        if (d == 128) return launch_tc<128, MODE_LEVEL, true>(Q, K, V, args, st);
+        return -2;
+    }
     if (d == 64) {
         if (level) return launch_tc<64, MODE_LEVEL>(Q, K, V, args, st);
         return dense ? launch_tc<64, MODE_DENSE>(Q, K, V, args, st) : launch_tc<64, MODE_CAUSAL>(Q, K, V, args, st);
@@ -1081,12 +1222,16 @@ int dispatch(int d, const void *Q, const void *K, const void *V, const TcArgs &a
 
 int launch_attn_tc(const Level &lv, const void *Q, const void *K, const void *V, int d, const int32_t *perm,
                    const int32_t *inv, const int32_t *S, int m, int64_t nodes_total, void *O, int out_dtype,
-                   float *lse, float *Opart, float *Lpart, int *status, cudaStream_t st, int64_t stall_ns) {
-    if ((d != 64 && d != 128) || lv.bp % 128 != 0 || lv.bp > kMaxBlock || m > kMaxSampleList ||
+                   float *lse, float *Opart, float *Lpart, int *status, cudaStream_t st, int64_t stall_ns,
+                   const int32_t *Srn, const float *lwrn) {
+    const bool rn = Srn != nullptr && m > 0;
+    if ((d != 64 && d != 128) || lv.bp % 128 != 0 || lv.bp > kMaxBlock || m > (rn ? kMaxSampleListRn : kMaxSampleList) ||
         lv.bh * lv.n >= (int64_t(1) << 31))
         return -2;
     TcArgs a{};
-    a.mode = MODE_LEVEL;
+    a.mode = rn ? MODE_LEVEL_RN : MODE_LEVEL;
+    a.Srn = rn ? Srn : nullptr;
+    a.lwrn = rn ? lwrn : nullptr;
     a.n = lv.n;
     a.bh = lv.bh;
     a.lv = lv;
@@ -1097,6 +1242,7 @@ int launch_attn_tc(const Level &lv, const void *Q, const void *K, const void *V,
     a.nodes_total = nodes_total;
     a.nb = lv.bp / kKC;
     a.ns = (m + kKC - 1) / kKC;
+    a.nr = rn ? a.ns : 0;
     a.tiles_per_block = lv.bp / 128;
     a.pairs_per_block = (a.tiles_per_block + 1) / 2;
     a.lw2 = m > 0 ? log2f(static_cast<float>(lv.seg_len) / static_cast<float>(m)) : 0.0f;

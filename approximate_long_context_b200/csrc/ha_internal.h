@@ -50,9 +50,12 @@ int launch_sort_pass(const Level &lv, const uint16_t *rank, SortPass ps, const i
 
 // SIMT attention of one level: for level 0 writes O (out dtype); for causal levels writes the parts
 // Opart[bh][n/2][d] (fp32, normalised) and Lpart[bh][n/2] (log normaliser) of this level.
+// Srn/lwrn (nullptr for uniform sampling): row-norm draws and their log weights, [bh][nodes_total][m]; when
+// given, the uniform samples S feed only the normaliser and the row-norm draws only the product with V.
 int launch_attn_simt(const Level &lv, const void *Q, const void *K, const void *V, int dtype, int d,
                      const int32_t *perm, const int32_t *inv, const int32_t *S, int m, int64_t nodes_total,
-                     void *O, int out_dtype, float *lse, float *Opart, float *Lpart, cudaStream_t st);
+                     void *O, int out_dtype, float *lse, float *Opart, float *Lpart, cudaStream_t st,
+                     const int32_t *Srn = nullptr, const float *lwrn = nullptr);
 
 // SIMT exact causal attention on leaves of `leaf` rows, merged with the parts of levels 1..L.
 int launch_causal_base_simt(const void *Q, const void *K, const void *V, int dtype, int64_t bh, int64_t n,
@@ -63,7 +66,8 @@ int launch_causal_base_simt(const void *Q, const void *K, const void *V, int dty
 int launch_attn_tc(const Level &lv, const void *Q, const void *K, const void *V, int d,
                    const int32_t *perm, const int32_t *inv, const int32_t *S, int m, int64_t nodes_total,
                    void *O, int out_dtype, float *lse, float *Opart, float *Lpart, int *status, cudaStream_t st,
-                   int64_t stall_ns = 0);
+                   int64_t stall_ns = 0, const int32_t *Srn = nullptr, const float *lwrn = nullptr);
+// Srn/lwrn (row-norm sampling, m <= 256; larger m returns -2): as for launch_attn_simt.
 int launch_causal_base_tc(const void *Q, const void *K, const void *V, int64_t bh, int64_t n, int d,
                           int64_t leaf, int levels, const float *Opart, const float *Lpart,
                           void *O, int out_dtype, int *status, cudaStream_t st, int64_t stall_ns = 0);
@@ -76,6 +80,27 @@ int launch_exact_tc(const void *Q, const void *K, const void *V, int64_t bh, int
 // inv: level-0 inverse permutations [bh][2][n]; scratch: 4 * bh * n floats.
 int launch_diagnostics(const void *Q, const void *K, int dtype, int64_t bh, int64_t n, int d, const int32_t *inv,
                        int64_t bp, int64_t first_col, float *scratch, double *out, cudaStream_t st);
+
+// Row-norm samples (ha_rownorm.cu): geometry of the sample sets of one call. Set (problem b, heap node k) has
+// m draws; its cumulative distribution lives at cdf[b * per_prob + offset of the set].
+struct RowNormGeom {
+    int64_t n;
+    int causal;
+    int depths;             // 1 (non-causal) or the causal levels L
+    int m;
+    int64_t nodes_total;    // sample sets per problem
+    int64_t slot0[33];      // first 2048-row chunk slot of each depth; slot0[depths] = slots
+    int64_t slots;          // chunk slots per problem
+    int64_t per_prob;       // cdf doubles per problem: n (non-causal) or L * n / 2
+};
+RowNormGeom rownorm_geometry(int64_t n, int causal, int levels, int m, int64_t nodes_total);
+// Squared norms nrm[bh][n] (fp32), chunk sums csum[bh][slots], cdf[bh][per_prob] (double), then the draws
+// S[bh][nodes_total][m] (row index local to the set's key rows, -1 when all its rows are zero) and their log
+// weights logw[bh][nodes_total][m] = log(total / (m ||v_j||^2)). Returns the kernels launched, -1 on error,
+// -2 if bh exceeds the grid's second dimension.
+int launch_rownorm_draws(const RowNormGeom &g, const void *V, int dtype, int d, int64_t bh, uint64_t seed,
+                         int64_t bh_offset, float *nrm, double *csum, double *cdf, int32_t *S, float *logw,
+                         cudaStream_t st);
 
 // ---- host-side draws (ha_draws.cpp) ----
 void draw_projection(uint64_t seed, int d, int r, float *P);

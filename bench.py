@@ -41,6 +41,11 @@ TRAFFIC = {
         "file": "ha_attn_tc.cu",
         "sha256": "a84a9f305c2ab9e21b2b7e7f88f78aa375e948dc8162dfa1f90f93b6c2f84901",
         "bytes": 8 * (205_855_232 + 46_793_728)},
+    # row-norm sampling (--sampling rownorm), 4-head capture scaled x8: 206.0 MB read + 44.6 MB written
+    ("attn", "long_bf16_n131072", "tc", "rownorm"): {
+        "file": "ha_attn_tc.cu",
+        "sha256": "6650df5df3dc9d8021e437523ad21193b7fced4b1f61325e8162791b32184d18",
+        "bytes": 8 * (206_016_256 + 44_589_056)},
     ("hash", "long_bf16_n131072", "tc"): {
         "file": "ha_hash.cu",
         "sha256": "4590cdf32028d354a14840822c657310cf7c55c4363a9d576b207e5aa9b08c08",
@@ -58,7 +63,7 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def algorithmic(w: wl.Workload, cls: str):
+def algorithmic(w: wl.Workload, cls: str, sampling: str = "uniform"):
     """Algorithmic work per launch of a kernel class: (bytes, flops)."""
     e = 2 if w.dtype == "bf16" else 4
     bh, n, d = w.bh, w.n, w.d
@@ -73,12 +78,17 @@ def algorithmic(w: wl.Workload, cls: str):
     if cls == "attn":
         N = n if not w.causal else n // 2                        # query rows per level launch
         flops = bh * 4.0 * N * d * (min(w.block, N if not w.causal else n) + w.m)
+        if sampling == "rownorm":                                # uniform samples: scores only; draws: both
+            flops += bh * 2.0 * N * d * w.m
         byts = bh * N * (3 * d * e + d * (e if not w.causal else 4) + 8)
         return byts, flops
     if cls == "causal_base":
         flops = bh * 2.0 * n * d * w.base
         byts = bh * n * (3 * d * e + d * e) + bh * n * levels * (d * 4 + 4) / 2
         return byts, flops
+    if cls == "draws":                                           # V read; norms written, read twice; cdf written
+        sets_rows = n if not w.causal else levels * n // 2
+        return bh * n * (d * e + 4) + bh * sets_rows * (4 * 2 + 8) + bh * w.m * 8, 0.0
     raise KeyError(cls)
 
 
@@ -159,7 +169,7 @@ def dist_setup():
     return world, rank, local
 
 
-def cpu_oracle_rate(w: wl.Workload, heads):
+def cpu_oracle_rate(w: wl.Workload, heads, sampling="uniform"):
     """Oracle time on full heads (all rows): returns (Mqueries*heads/s, seconds, threads)."""
     import oracle
     oracle.build()
@@ -167,7 +177,7 @@ def cpu_oracle_rate(w: wl.Workload, heads):
     t0 = time.perf_counter()
     for i, h in enumerate(heads):
         oracle.forward(wl.as_f32(Qh[i]), wl.as_f32(Kh[i]), wl.as_f32(Vh[i]), block=w.block, m=w.m, r=w.r,
-                       causal=w.causal, base=w.base, seed=w.algo_seed, bh=h)
+                       causal=w.causal, base=w.base, seed=w.algo_seed, bh=h, sampling=sampling)
     dt = time.perf_counter() - t0
     return len(heads) * w.n / dt / 1e6, dt, oracle.num_threads()
 
@@ -183,7 +193,8 @@ def run_reference(args, w: wl.Workload):
     Qf, Kf, Vf = wl.as_f32(Qh[0]), wl.as_f32(Kh[0]), wl.as_f32(Vh[0])
 
     def step():
-        oracle.forward(Qf, Kf, Vf, block=w.block, m=w.m, r=w.r, causal=w.causal, base=w.base, seed=w.algo_seed, bh=0)
+        oracle.forward(Qf, Kf, Vf, block=w.block, m=w.m, r=w.r, causal=w.causal, base=w.base, seed=w.algo_seed, bh=0,
+                       sampling=args.sampling)
 
     for _ in range(args.warmup):
         step()
@@ -197,7 +208,7 @@ def run_reference(args, w: wl.Workload):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_of(w),
+        "config": config_of(w, args.sampling),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -229,11 +240,14 @@ def approx_error(Qf, Kf, Vf, Of, causal: bool, nrows: int = 256, seed: int = 7):
             "rows": int(len(rows)), "head": 0, "vs": "exact softmax attention (float64 numpy, sampled rows)"}
 
 
-def config_of(w: wl.Workload):
-    return {"workload": w.name, "batch": w.batch, "heads": w.heads, "n": w.n, "d": w.d, "block": w.block, "m": w.m,
-            "r": w.r, "causal": w.causal, "causal_base": w.base if w.causal else None, "input_dtype": w.dtype,
-            "parallelism": "independent (batch, head) problems per GPU; no collective",
-            "l2": "inputs larger than L2, no flush" if 3 * w.bh * w.n * w.d * 2 > 2 * L2_BYTES else "L2 flushed"}
+def config_of(w: wl.Workload, sampling: str = "uniform"):
+    c = {"workload": w.name, "batch": w.batch, "heads": w.heads, "n": w.n, "d": w.d, "block": w.block, "m": w.m,
+         "r": w.r, "causal": w.causal, "causal_base": w.base if w.causal else None, "input_dtype": w.dtype,
+         "parallelism": "independent (batch, head) problems per GPU; no collective",
+         "l2": "inputs larger than L2, no flush" if 3 * w.bh * w.n * w.d * 2 > 2 * L2_BYTES else "L2 flushed"}
+    if sampling != "uniform":
+        c["sampling"] = sampling
+    return c
 
 
 def run_ours(args, w: wl.Workload):
@@ -276,7 +290,7 @@ def run_ours(args, w: wl.Workload):
 
     ha = binding.HyperAttention(local)
     ha.set_options(dtype=w.dtype, batch=w.batch, causal_base=w.base or 4096, stream=stream.cuda_stream,
-                   kernel=args.kernel, bh_offset=sh.offset)
+                   kernel=args.kernel, bh_offset=sh.offset, sampling=args.sampling)
     kw = dict(n=w.n, d=w.d, heads=w.heads, block=w.block, m=w.m, r=w.r, causal=w.causal, seed=w.algo_seed)
 
     def step():
@@ -370,7 +384,7 @@ def run_ours(args, w: wl.Workload):
     nlev = int(round(np.log2(w.n // w.base))) if (w.causal and w.n > w.base) else (0 if w.causal else 1)
     groups = nlev if dom in ("sort", "attn") else 1
     avg_ms = dom_ms / (args.steps * groups)
-    byts, flops = algorithmic(w, dom)
+    byts, flops = algorithmic(w, dom, args.sampling)
     if flops > 0 and dom in ("attn", "causal_base"):
         # the binding roof is the one with the larger ideal time: algorithmic bytes at HBM peak or FLOPs at the
         # compute peak (tensor for the tcgen05 kernels, FP32 ALU for the SIMT ones)
@@ -387,7 +401,7 @@ def run_ours(args, w: wl.Workload):
         bound, peak, unit = "hbm", peaks["hbm_gbs"], "GB/s"
         achieved = byts / (avg_ms * 1e-3) / 1e9
     traffic = None
-    tr = TRAFFIC.get((dom, w.name, family))
+    tr = TRAFFIC.get((dom, w.name, family) + ((args.sampling,) if args.sampling != "uniform" else ()))
     if tr is not None:
         src = os.path.join(ROOT, "approximate_long_context_b200", "csrc", tr["file"])
         if os.path.exists(src) and hashlib.sha256(open(src, "rb").read()).hexdigest() == tr["sha256"]:
@@ -401,7 +415,7 @@ def run_ours(args, w: wl.Workload):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         heads = list(range(min(args.cpu_heads, w.bh)))
-        rate, secs, cores = cpu_oracle_rate(w, heads)
+        rate, secs, cores = cpu_oracle_rate(w, heads, args.sampling)
         cpu = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": f"{len(heads)} of {w.bh} heads, all {w.n} query rows ({secs:.1f} s)"}
 
@@ -410,7 +424,7 @@ def run_ours(args, w: wl.Workload):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded Gaussian Q/K/V, planted heavy keys)",
-            "config": config_of(w),
+            "config": config_of(w, args.sampling),
             "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                          "frac": achieved / peak, "traffic": traffic, "kernel": dom,
                          "kernel_ms_per_launch": avg_ms, "peak_source": peak_src + (" burst" if bound == "tensor" else ""),
@@ -440,6 +454,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=wl.HEADLINE, choices=sorted(wl.WORKLOADS))
     ap.add_argument("--kernel", default="auto", choices=["auto", "simt", "tc"])
+    ap.add_argument("--sampling", default="uniform", choices=["uniform", "rownorm"],
+                    help="samples of the product with V: the uniform ones, or rows of V by squared norm")
     ap.add_argument("--cpu-heads", type=int, default=32)
     ap.add_argument("--heads", type=int, default=0,
                     help="run the workload with this many heads instead of its own (small profiler captures)")

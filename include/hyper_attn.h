@@ -56,6 +56,17 @@ typedef enum { HA_DTYPE_BF16 = 0, HA_DTYPE_FP32 = 1 } ha_dtype;
  * fp32 inputs. SIMT: SIMT fp32 kernels for any input type. TC: tensor-core kernels (bf16 only). */
 typedef enum { HA_KERNEL_AUTO = 0, HA_KERNEL_SIMT = 1, HA_KERNEL_TC = 2 } ha_kernel;
 
+/* How the sampled part of the product with V is estimated ("HyperAttention: Long-context Attention in
+ * Near-Linear Time", research-map summary, "Approach").
+ * UNIFORM: the m uniform column samples of the normaliser also serve the product with V (weight N/m).
+ * ROWNORM: the normaliser keeps the uniform samples; the product with V takes m draws with replacement,
+ *   row j with probability p_j = ||v_j||^2 / sum ||v||^2 over the problem's key rows, weight 1/(m p_j).
+ *   The squared norms are sequential fp32 multiply-adds, the draws Philox4x64-10 under key (seed, 3) at
+ *   counter (t/4, node, bh, 0), word t mod 4, u = (w >> 11) 2^-53, the smallest j whose cumulative sum
+ *   exceeds u times the total; all of it runs on the device. The tensor-core kernels take m <= 256 (bf16);
+ *   beyond that AUTO falls back to the SIMT kernels and HA_KERNEL_TC returns HA_ERR_UNSUPPORTED. */
+typedef enum { HA_SAMPLING_UNIFORM = 0, HA_SAMPLING_ROWNORM = 1 } ha_sampling;
+
 typedef struct {
     int dtype;            /* ha_dtype of Q, K, V. Default HA_DTYPE_BF16. */
     int out_dtype;        /* ha_dtype of O, or -1 for "same as dtype". Default -1. */
@@ -69,11 +80,12 @@ typedef struct {
                              of local problem i are those of problem bh_offset + i, so a run split over
                              several calls or GPUs (each taking a contiguous range of problems) gives the
                              same result as one call over all problems. Default 0. */
-    int test_stall_ms;    /* Test hook for the failure path, 0..1000. When > 0, the tensor-core attention
-                             kernel's first softmax wait targets a barrier that nothing ever completes and
-                             gives up after this many milliseconds: every role of the kernel then stops,
-                             the output is undefined, and hyper_attn_status reports HA_ERR_TIMEOUT. The
-                             device stays usable. Default 0 (off). */
+    int test_stall_ms;    /* Test hook for the failure path, 0..1000. When > 0, the tensor-core level kernel
+                             (uniform sampling; a separate instance of it) makes its first softmax wait target a
+                             barrier that nothing ever completes and give up after this many milliseconds:
+                             every role of the kernel then stops, the output is undefined, and
+                             hyper_attn_status reports HA_ERR_TIMEOUT. The device stays usable. Default 0. */
+    int sampling;         /* ha_sampling of the product with V. Default HA_SAMPLING_UNIFORM. */
 } ha_options;
 
 /* Create a handle bound to CUDA device `device`. The handle owns a grow-only device workspace (ranks,
@@ -175,7 +187,9 @@ typedef enum {
     HA_DBG_NEAR = 1,   /* uint8  [bh][2][n]: 1 when some projection of the row is below 1e-4 * ||row||  */
     HA_DBG_PERM = 2,   /* int32  [bh][nodes_l][2][N_l]: sorted position -> local row, Q then K segment   */
     HA_DBG_INV = 3,    /* int32  [bh][nodes_l][2][N_l]: local row -> sorted position                     */
-    HA_DBG_LSE = 4     /* float  [bh][n]: log of the estimated normaliser of each query row (non-causal) */
+    HA_DBG_LSE = 4,    /* float  [bh][n]: log of the estimated normaliser of each query row (non-causal) */
+    HA_DBG_RN_S = 5,   /* int32  [bh][nodes][m]: row-norm draws, row index local to the set's key rows    */
+    HA_DBG_RN_LOGW = 6 /* float  [bh][nodes][m]: their log weights log(1 / (m p_j))                       */
 } ha_debug_what;
 HA_API int hyper_attn_debug_copy(hyper_attn_t h, int what, int level, void *host_dst, size_t bytes);
 
@@ -189,7 +203,8 @@ typedef enum {
     HA_KC_SORT = 1,        /* counting-sort passes (count, scan, scatter) */
     HA_KC_ATTN = 2,        /* block + sampled attention of one level, including the gather and the merge */
     HA_KC_CAUSAL_BASE = 3, /* exact causal leaves and the final log-space merge */
-    HA_KC_COUNT = 4
+    HA_KC_DRAWS = 4,       /* row-norm draws on the device (norms, cumulative sums, draws) */
+    HA_KC_COUNT = 5
 } ha_kernel_class;
 
 /* enable = 1: record a CUDA event pair on the handle's stream around every kernel class launch of the

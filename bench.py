@@ -36,11 +36,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # taken from is unchanged (sha256 of the file at capture time).
 TRAFFIC = {
     # 4-head capture of the 32-head workload (the full one is too large for a multi-pass capture), scaled x8
-    # by the rows processed: attention 205.9 MB read + 46.8 MB written per 4-head launch; hash 134.2 + 6.2 MB.
+    # by the rows processed: attention 205.8 MB read + 42.9 MB written per 4-head launch; hash 134.2 + 6.2 MB.
     ("attn", "long_bf16_n131072", "tc"): {
         "file": "ha_attn_tc.cu",
-        "sha256": "a84a9f305c2ab9e21b2b7e7f88f78aa375e948dc8162dfa1f90f93b6c2f84901",
-        "bytes": 8 * (205_855_232 + 46_793_728)},
+        "sha256": "6650df5df3dc9d8021e437523ad21193b7fced4b1f61325e8162791b32184d18",
+        "bytes": 8 * (205_804_288 + 42_924_800)},
     # row-norm sampling (--sampling rownorm), 4-head capture scaled x8: 206.0 MB read + 44.6 MB written
     ("attn", "long_bf16_n131072", "tc", "rownorm"): {
         "file": "ha_attn_tc.cu",

@@ -55,11 +55,11 @@ KW = dict(block=64, m=32, r=6, causal=False, seed=77)
 DATA_SEED = 0xABC
 
 
-def _run_problem(Q, K, V, g, ora):
-    return ora.forward(wl.as_f32(Q), wl.as_f32(K), wl.as_f32(V), bh=g, **KW)["O"]
+def _run_problem(Q, K, V, g, ora, sampling="uniform"):
+    return ora.forward(wl.as_f32(Q), wl.as_f32(K), wl.as_f32(V), bh=g, sampling=sampling, **KW)["O"]
 
 
-def _rank_main(rank, world, port, out_dir):
+def _rank_main(rank, world, port, out_dir, sampling):
     import torch.distributed as dist
     import oracle
     os.environ["MASTER_ADDR"] = "127.0.0.1"
@@ -70,7 +70,7 @@ def _rank_main(rank, world, port, out_dir):
         s = shard.shard_problems(G, world, rank)
         heads = range(s.offset, s.offset + s.count)
         Q, K, V = wl.make_inputs(N, D, G, data_seed=DATA_SEED, dtype="fp32", heads=heads)
-        outs = [_run_problem(Q[i], K[i], V[i], g, oracle) for i, g in enumerate(heads)]
+        outs = [_run_problem(Q[i], K[i], V[i], g, oracle, sampling) for i, g in enumerate(heads)]
         local = np.stack(outs) if outs else np.zeros((0, N, D))
         gathered = [None] * world
         dist.all_gather_object(gathered, (s.offset, local))
@@ -89,15 +89,18 @@ def _free_port():
         return sk.getsockname()[1]
 
 
-def test_two_gloo_ranks_equal_one_run(tmp_path, ora):
+@pytest.mark.parametrize("sampling", ["uniform", "rownorm"])
+def test_two_gloo_ranks_equal_one_run(tmp_path, ora, sampling):
+    """Both samplings key their draws by the global problem index (the row-norm draws also by the problem's own
+    value rows), so split runs equal one run."""
     import torch.multiprocessing as mp
     world = 2
-    mp.start_processes(_rank_main, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True,
+    mp.start_processes(_rank_main, args=(world, _free_port(), str(tmp_path), sampling), nprocs=world, join=True,
                        start_method="spawn")
     job = np.load(tmp_path / "job.npy")
     assert np.load(tmp_path / "tmax.npy")[0] == 2.5           # the slowest rank's time
     Q, K, V = wl.make_inputs(N, D, G, data_seed=DATA_SEED, dtype="fp32")
-    whole = np.stack([_run_problem(Q[g], K[g], V[g], g, ora) for g in range(G)])
+    whole = np.stack([_run_problem(Q[g], K[g], V[g], g, ora, sampling) for g in range(G)])
     assert job.shape == whole.shape
     assert np.array_equal(job, whole)
 
@@ -106,6 +109,7 @@ def test_problem_index_keys_the_draws(ora):
     """A rank that ignored its offset (keying its draws by local index) would give a different result:
     the check above can fail."""
     Q, K, V = wl.make_inputs(N, D, 1, data_seed=DATA_SEED, dtype="fp32", heads=[3])
-    a = _run_problem(Q[0], K[0], V[0], 3, ora)
-    b = _run_problem(Q[0], K[0], V[0], 0, ora)
-    assert not np.array_equal(a, b)
+    for sampling in ("uniform", "rownorm"):
+        a = _run_problem(Q[0], K[0], V[0], 3, ora, sampling)
+        b = _run_problem(Q[0], K[0], V[0], 0, ora, sampling)
+        assert not np.array_equal(a, b)

@@ -74,6 +74,14 @@ def _load():
                                     ctypes.c_uint64, ctypes.c_int64, ctypes.POINTER(ctypes.c_double),
                                     ctypes.POINTER(ctypes.c_double)]
     lib.ora_diagnostics.restype = ctypes.c_int
+    lib.ora_weights.argtypes = [_f32p, _f32p, _f32p, ctypes.c_int64, ctypes.c_int, ctypes.c_int64, ctypes.c_int,
+                                ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_uint64, ctypes.c_int64,
+                                ctypes.c_int, _f64p, _f64p]
+    lib.ora_weights.restype = ctypes.c_int
+    lib.ora_backward.argtypes = [_f32p, _f32p, _f32p, _f32p, ctypes.c_int64, ctypes.c_int, ctypes.c_int64,
+                                 ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_uint64,
+                                 ctypes.c_int64, ctypes.c_int, _f64p, _f64p, _f64p, _f64p, _f64p]
+    lib.ora_backward.restype = ctypes.c_int
     lib.ora_num_threads.argtypes = []
     lib.ora_num_threads.restype = ctypes.c_int
     _lib = lib
@@ -198,6 +206,37 @@ def diagnostics(Q, K, *, block: int, r: int, seed: int, first_col: int = 0):
     _check(_load().ora_diagnostics(Q, K, n, d, block, r, seed, first_col, ctypes.byref(alpha), ctypes.byref(kappa)),
            "diagnostics")
     return alpha.value, kappa.value
+
+
+def weights(Q, K, V, *, block: int, m: int, r: int, causal: bool, seed: int, bh: int = 0, base: int = 0,
+            sampling: str = "uniform"):
+    """Dense (n, n) numerator and normaliser weights (Wn, Wd) of one problem: O = (Wn o E) V / rowsum(Wd o E),
+    E = exp(Q K^T) (see oracle.c). For small n."""
+    Q = np.ascontiguousarray(Q, np.float32)
+    K = np.ascontiguousarray(K, np.float32)
+    V = np.ascontiguousarray(V, np.float32)
+    n, d = Q.shape
+    Wn = np.zeros((n, n), np.float64)
+    Wd = np.zeros((n, n), np.float64)
+    _check(_load().ora_weights(Q, K, V, n, d, block, m, r, int(causal), base, seed, bh, SAMPLING[sampling], Wn, Wd),
+           "weights")
+    return Wn, Wd
+
+
+def backward(Q, K, V, dO, *, block: int, m: int, r: int, causal: bool, seed: int, bh: int = 0, base: int = 0,
+             sampling: str = "uniform"):
+    """Gradients of sum(dO * O) of one problem with respect to Q, K, V (float64, (n, d) each), the sort and the
+    draws held fixed; also O and the log normaliser L. Dense: for small n."""
+    Q = np.ascontiguousarray(Q, np.float32)
+    K = np.ascontiguousarray(K, np.float32)
+    V = np.ascontiguousarray(V, np.float32)
+    dO = np.ascontiguousarray(dO, np.float32)
+    n, d = Q.shape
+    out = {k: np.zeros((n, d), np.float64) for k in ("dQ", "dK", "dV", "O")}
+    out["L"] = np.zeros(n, np.float64)
+    _check(_load().ora_backward(Q, K, V, dO, n, d, block, m, r, int(causal), base, seed, bh, SAMPLING[sampling],
+                                out["dQ"], out["dK"], out["dV"], out["O"], out["L"]), "backward")
+    return out
 
 
 def exact_attention(Q, K, V, *, causal: bool, rows=None) -> np.ndarray:

@@ -1,5 +1,5 @@
 /*
- * oracle.c -- plain, slow CPU reference of the HyperAttention forward pass.
+ * oracle.c -- plain, slow CPU reference of the HyperAttention forward pass and its gradients.
  *
  * TEST INFRASTRUCTURE. Only the test suite, the package smoke check and the benchmark's CPU-baseline
  * leg load this library. It shares no code, header, table or helper with the CUDA library and it
@@ -688,6 +688,169 @@ int ora_diagnostics(const float *Q, const float *K, int64_t n, int d, int64_t bl
     free(P); free(rq); free(rk); free(fl); free(pq); free(pk); free(posq); free(posk);
     free(m); free(D); free(logR); free(col);
     return ORA_OK;
+}
+
+/*
+ * Dense weights of one problem, for the backward pass. The forward estimate of every row q is a weighted
+ * softmax over the keys: O_q = sum_k Wn[q][k] e^{s_qk} v_k / sum_k Wd[q][k] e^{s_qk}, s_qk = q . k, where
+ *   - a key in q's sortLSH block (of a level's subproblem, or of q's exact causal leaf) has Wn = Wd = 1;
+ *   - a uniform sample outside the block has Wd = N/m, and Wn = N/m unless the product with V is row-norm
+ *     sampled;
+ *   - with row-norm sampling, every draw outside the block adds 1/(m p_j) to Wn (draws may repeat).
+ * The log-space merges of the causal recursion combine the parts into exactly this form, because the parts'
+ * key sets are disjoint. The weights follow the same steps as ora_forward_sampling (same projection, ranks,
+ * sorts and draws); the sort permutation and the draws are constants of the forward pass.
+ */
+static int sub_weights(int64_t n, int64_t N, int64_t q0, int64_t k0, const uint16_t *rq, const uint16_t *rk,
+                       int64_t block, const int32_t *S, int m, const int32_t *Srn, const double *lwrn,
+                       double *Wn, double *Wd)
+{
+    int64_t bp = block < N ? block : N;
+    if (bp <= 0 || N % bp != 0) return ORA_EINVAL;
+    int32_t *permQ = (int32_t *)malloc(sizeof(int32_t) * (size_t)N);
+    int32_t *permK = (int32_t *)malloc(sizeof(int32_t) * (size_t)N);
+    int64_t *posQ = (int64_t *)malloc(sizeof(int64_t) * (size_t)N);
+    int64_t *posK = (int64_t *)malloc(sizeof(int64_t) * (size_t)N);
+    int rc = (!permQ || !permK || !posQ || !posK) ? ORA_ENOMEM : ORA_OK;
+    if (rc == ORA_OK) rc = ora_sort_segment(rq, N, permQ);
+    if (rc == ORA_OK) rc = ora_sort_segment(rk, N, permK);
+    if (rc == ORA_OK) {
+        for (int64_t p = 0; p < N; ++p) { posQ[permQ[p]] = p; posK[permK[p]] = p; }
+        const double w = m > 0 ? (double)N / (double)m : 0.0;
+        for (int64_t q = 0; q < N; ++q) {
+            const int64_t i = posQ[q] / bp;
+            double *wn = Wn + (q0 + q) * n + k0, *wd = Wd + (q0 + q) * n + k0;
+            for (int64_t j = 0; j < bp; ++j) {
+                const int64_t k = permK[i * bp + j];
+                wn[k] += 1.0;
+                wd[k] += 1.0;
+            }
+            for (int u = 0; u < m; ++u) {
+                const int64_t k = S[u];
+                if (posK[k] / bp == i) continue;
+                wd[k] += w;
+                if (!Srn) wn[k] += w;
+            }
+            for (int u = 0; Srn && u < m; ++u) {
+                const int64_t k = Srn[u];
+                if (k < 0 || posK[k] / bp == i) continue;
+                wn[k] += exp(lwrn[u]);
+            }
+        }
+    }
+    free(permQ); free(permK); free(posQ); free(posK);
+    return rc;
+}
+
+int ora_weights(const float *Q, const float *K, const float *V, int64_t n, int d, int64_t block, int m, int r,
+                int causal, int64_t base, uint64_t seed, int64_t bh, int sampling, double *Wn, double *Wd)
+{
+    if (sampling != 0 && sampling != 1) return ORA_EINVAL;
+    if (n <= 0 || d <= 0 || block <= 0 || m < 0 || r < 0 || r > 16) return ORA_EINVAL;
+    if (causal && !valid_causal_shape(n, base)) return ORA_EINVAL;
+    int rc = ORA_OK;
+    float *P = (float *)malloc(sizeof(float) * (size_t)(d * (r > 0 ? r : 1)));
+    uint16_t *rank = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)(2 * n));
+    uint8_t *near = (uint8_t *)malloc((size_t)(2 * n));
+    int32_t *S = (int32_t *)malloc(sizeof(int32_t) * (size_t)(m > 0 ? m : 1));
+    int32_t *Srn = (int32_t *)malloc(sizeof(int32_t) * (size_t)(m > 0 ? m : 1));
+    double *lw = (double *)malloc(sizeof(double) * (size_t)(m > 0 ? m : 1));
+    if (!P || !rank || !near || !S || !Srn || !lw) { rc = ORA_ENOMEM; goto out; }
+    memset(Wn, 0, sizeof(double) * (size_t)(n * n));
+    memset(Wd, 0, sizeof(double) * (size_t)(n * n));
+    ora_draw_projection(seed, d, r, P);
+    ora_hash_rows(Q, n, d, P, r, rank, near);
+    ora_hash_rows(K, n, d, P, r, rank + n, near + n);
+    if (!causal) {
+        if (m > n) { rc = ORA_EINVAL; goto out; }
+        rc = ora_draw_samples(seed, bh, 1, n, m, S);
+        if (rc == ORA_OK && sampling) rc = ora_draw_rownorm(seed, bh, 1, V, n, d, m, Srn, lw);
+        if (rc == ORA_OK)
+            rc = sub_weights(n, n, 0, 0, rank, rank + n, block, S, m, sampling ? Srn : NULL, lw, Wn, Wd);
+        goto out;
+    }
+    {
+        const int64_t leaf = base < n ? base : n;
+        for (int64_t q = 0; q < n; ++q)
+            for (int64_t k = q - q % leaf; k <= q; ++k) { Wn[q * n + k] = 1.0; Wd[q * n + k] = 1.0; }
+        for (int64_t len = n; len > leaf && rc == ORA_OK; len >>= 1) {
+            const int64_t half = len / 2, nodes = n / len;
+            if (m > half) { rc = ORA_EINVAL; break; }
+            for (int64_t j = 0; j < nodes && rc == ORA_OK; ++j) {
+                const int64_t s0 = j * len, node = nodes + j;
+                rc = ora_draw_samples(seed, bh, node, half, m, S);
+                if (rc == ORA_OK && sampling) rc = ora_draw_rownorm(seed, bh, node, V + s0 * d, half, d, m, Srn, lw);
+                if (rc == ORA_OK)
+                    rc = sub_weights(n, half, s0 + half, s0, rank + s0 + half, rank + n + s0, block, S, m,
+                                     sampling ? Srn : NULL, lw, Wn, Wd);
+            }
+        }
+    }
+out:
+    free(P); free(rank); free(near); free(S); free(Srn); free(lw);
+    return rc;
+}
+
+/*
+ * Backward pass of one problem: the gradients of sum_q dO_q . O_q with respect to Q, K and V, with the sort
+ * permutations and the draws held fixed (they are constants of the forward pass). With the dense weights
+ * above, E_qk = e^{s_qk - L_q} where L_q = log sum_k Wd[q][k] e^{s_qk}, and g_q = dO_q . O_q:
+ *   dV_k = sum_q Wn[q][k] E_qk dO_q,
+ *   dS_qk = E_qk (Wn[q][k] (dO_q . v_k) - Wd[q][k] g_q),
+ *   dQ_q = sum_k dS_qk k_k,   dK_k = sum_q dS_qk q_q.
+ * (O_q = N_q / D_q with N_q = sum_k Wn e^{s} v_k and D_q = sum_k Wd e^{s}; differentiate the quotient.) Double
+ * precision, dense over all (q, k): for small n. Also returns O and L.
+ */
+int ora_backward(const float *Q, const float *K, const float *V, const float *dO, int64_t n, int d, int64_t block,
+                 int m, int r, int causal, int64_t base, uint64_t seed, int64_t bh, int sampling,
+                 double *dQ, double *dK, double *dV, double *O, double *L)
+{
+    double *Wn = (double *)malloc(sizeof(double) * (size_t)(n * n));
+    double *Wd = (double *)malloc(sizeof(double) * (size_t)(n * n));
+    double *sc = (double *)malloc(sizeof(double) * (size_t)n);
+    if (!Wn || !Wd || !sc) { free(Wn); free(Wd); free(sc); return ORA_ENOMEM; }
+    int rc = ora_weights(Q, K, V, n, d, block, m, r, causal, base, seed, bh, sampling, Wn, Wd);
+    if (rc == ORA_OK) {
+        memset(dQ, 0, sizeof(double) * (size_t)(n * d));
+        memset(dK, 0, sizeof(double) * (size_t)(n * d));
+        memset(dV, 0, sizeof(double) * (size_t)(n * d));
+        for (int64_t q = 0; q < n; ++q) {
+            const double *wn = Wn + q * n, *wd = Wd + q * n;
+            double mx = -INFINITY;
+            for (int64_t k = 0; k < n; ++k) {
+                sc[k] = (wn[k] != 0.0 || wd[k] != 0.0) ? dot_fd(Q + q * d, K + k * d, d) : -INFINITY;
+                if (sc[k] > mx) mx = sc[k];
+            }
+            double den = 0.0;
+            double *o = O + q * d;
+            for (int c = 0; c < d; ++c) o[c] = 0.0;
+            for (int64_t k = 0; k < n; ++k) {
+                if (sc[k] == -INFINITY) continue;
+                const double e = exp(sc[k] - mx);
+                den += wd[k] * e;
+                for (int c = 0; c < d; ++c) o[c] += wn[k] * e * (double)V[k * d + c];
+            }
+            for (int c = 0; c < d; ++c) o[c] /= den;
+            const double Lq = mx + log(den);
+            L[q] = Lq;
+            double g = 0.0;
+            for (int c = 0; c < d; ++c) g += (double)dO[q * d + c] * o[c];
+            for (int64_t k = 0; k < n; ++k) {
+                if (sc[k] == -INFINITY) continue;
+                const double E = exp(sc[k] - Lq);
+                double dov = 0.0;
+                for (int c = 0; c < d; ++c) dov += (double)dO[q * d + c] * (double)V[k * d + c];
+                const double ds = E * (wn[k] * dov - wd[k] * g);
+                for (int c = 0; c < d; ++c) {
+                    dV[k * d + c] += wn[k] * E * (double)dO[q * d + c];
+                    dQ[q * d + c] += ds * (double)K[k * d + c];
+                    dK[k * d + c] += ds * (double)Q[q * d + c];
+                }
+            }
+        }
+    }
+    free(Wn); free(Wd); free(sc);
+    return rc;
 }
 
 int ora_num_threads(void)

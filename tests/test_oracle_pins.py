@@ -539,3 +539,93 @@ def test_rownorm_numerator_unbiased(ora):
     se = est.std(axis=0, ddof=1) / np.sqrt(T)
     z = (est.mean(axis=0) - ref) / se
     assert np.abs(z).max() < 5.0, np.abs(z).max()
+
+
+# ---------------------------------------------------------------- backward pass
+# The gradients of sum(dO * O) with the sort and the draws held fixed. Pinned by finite differences of the
+# (separately pinned) forward, by exact attention's gradient where the method reduces to it, and by two
+# identities of a weighted softmax that hold for any weights.
+
+def _loss(ora, Q, K, V, dO, kw):
+    return float((ora.forward(Q, K, V, **kw)["O"] * dO.astype(np.float64)).sum())
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("sampling", ["uniform", "rownorm"])
+def test_weights_reproduce_forward(ora, causal, sampling):
+    n, d = 256, 16
+    Q, K, V = rand_qkv(n, d, 61)
+    kw = dict(block=16, m=12, r=4, causal=causal, base=32, seed=5, bh=2, sampling=sampling)
+    Wn, Wd = ora.weights(Q, K, V, **kw)
+    S = Q.astype(np.float64) @ K.astype(np.float64).T
+    mx = np.where((Wn > 0) | (Wd > 0), S, -np.inf).max(axis=1, keepdims=True)
+    E = np.exp(S - mx)
+    ref = ora.forward(Q, K, V, **kw)
+    np.testing.assert_allclose((Wn * E) @ V.astype(np.float64) / (Wd * E).sum(1, keepdims=True), ref["O"],
+                               rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(mx[:, 0] + np.log((Wd * E).sum(1)), ref["L"], rtol=0, atol=1e-10)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("sampling,which", [("uniform", "Q"), ("uniform", "K"), ("uniform", "V"),
+                                            ("rownorm", "Q"), ("rownorm", "K")])
+def test_backward_finite_differences(ora, causal, sampling, which):
+    """Central differences of the forward along a random direction. With row-norm sampling V also sets the
+    draws and their weights, which the backward holds fixed, so V is checked by the identity test below."""
+    n, d, eps = 128, 16, 1e-3
+    Q, K, V = rand_qkv(n, d, 62)
+    rng = np.random.default_rng(7)
+    dO = rng.standard_normal((n, d)).astype(np.float32)
+    kw = dict(block=16, m=12, r=4, causal=causal, base=32, seed=9, bh=0, sampling=sampling)
+    g = ora.backward(Q, K, V, dO, **kw)["d" + which]
+    X = {"Q": Q, "K": K, "V": V}[which]
+    E = rng.standard_normal(X.shape)
+    if which in "QK":   # leave alone the rows with a projection close enough to zero to change sign
+        proj = X.astype(np.float64) @ ora.draw_projection(9, d, 4).astype(np.float64)
+        E[np.abs(proj).min(axis=1) < 0.05] = 0.0
+    Xp = (X + eps * E).astype(np.float32)
+    Xm = (X - eps * E).astype(np.float32)
+    args = lambda Y: [Y if nm == which else {"Q": Q, "K": K, "V": V}[nm] for nm in "QKV"]
+    rank0 = ora.forward(Q, K, V, **kw)["rank"]
+    for Y in (Xp, Xm):   # the perturbation must not move a row to another bucket
+        assert np.array_equal(ora.forward(*args(Y), **kw)["rank"], rank0)
+    fd = _loss(ora, *args(Xp), dO, kw) - _loss(ora, *args(Xm), dO, kw)
+    an = float((g * (Xp.astype(np.float64) - Xm.astype(np.float64))).sum())
+    assert abs(fd - an) <= 1e-5 * abs(an) + 1e-9, (fd, an)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_reduces_to_exact_attention(ora, causal):
+    """One block covering every key (non-causal), or one exact causal leaf (c >= n): the estimate is exact
+    softmax attention, and so is its gradient, written here from the definition."""
+    n, d = 128, 16
+    Q, K, V = rand_qkv(n, d, 63)
+    dO = np.random.default_rng(8).standard_normal((n, d)).astype(np.float32)
+    out = ora.backward(Q, K, V, dO, block=n, m=16, r=4, causal=causal, base=n, seed=2)
+    Qd, Kd, Vd, G = (x.astype(np.float64) for x in (Q, K, V, dO))
+    S = Qd @ Kd.T
+    if causal:
+        S = np.where(np.tril(np.ones((n, n), bool)), S, -np.inf)
+    P = np.exp(S - S.max(1, keepdims=True))
+    P /= P.sum(1, keepdims=True)
+    dP = G @ Vd.T
+    dS = P * (dP - (dP * P).sum(1, keepdims=True))
+    np.testing.assert_allclose(out["dV"], P.T @ G, rtol=1e-9, atol=1e-12)
+    np.testing.assert_allclose(out["dQ"], dS @ Kd, rtol=1e-9, atol=1e-12)
+    np.testing.assert_allclose(out["dK"], dS.T @ Qd, rtol=1e-9, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("sampling", ["uniform", "rownorm"])
+def test_backward_identities(ora, causal, sampling):
+    """For any weighted softmax: shifting every key by the same vector leaves each row's output unchanged,
+    so the key gradients sum to zero; and O is linear in V at fixed weights, so sum(dV * V) = sum(dO * O)."""
+    n, d = 256, 16
+    Q, K, V = rand_qkv(n, d, 64)
+    dO = np.random.default_rng(9).standard_normal((n, d)).astype(np.float32)
+    out = ora.backward(Q, K, V, dO, block=16, m=12, r=4, causal=causal, base=32, seed=4, bh=1, sampling=sampling)
+    scale = np.abs(out["dK"]).sum(0).max()
+    assert np.abs(out["dK"].sum(0)).max() <= 1e-12 * scale + 1e-13
+    lhs = float((out["dV"] * V.astype(np.float64)).sum())
+    rhs = float((out["O"] * dO.astype(np.float64)).sum())
+    assert lhs == pytest.approx(rhs, rel=1e-12, abs=1e-12)

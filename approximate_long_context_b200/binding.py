@@ -26,7 +26,7 @@ EXPORTS = [
     "hyper_attn_status", "hyper_attn_last_launch_count", "hyper_attn_last_error", "hyper_attn_destroy",
     "hyper_attn_version", "hyper_attn_profile", "hyper_attn_profile_read",
     "hyper_attn_last_kernel", "hyper_attn_forward_noalloc", "hyper_attn_exact",
-    "hyper_attn_diagnostics",
+    "hyper_attn_diagnostics", "hyper_attn_backward",
 ]
 KERNEL_CLASSES = ["hash", "sort", "attn", "causal_base", "draws"]
 
@@ -72,6 +72,7 @@ def lib():
     L.hyper_attn_forward_host.argtypes = fwd
     L.hyper_attn_exact.argtypes = [vp, vp, vp, vp, vp, i64, ci, ci, ci]
     L.hyper_attn_diagnostics.argtypes = [vp, vp, vp, i64, ci, ci, ci, ci, u64, i64, vp, vp]
+    L.hyper_attn_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i64, ci, ci, ci, ci, ci, ci, u64]
     L.hyper_attn_draw.argtypes = [u64, ci, ci, i64, i64, ci, ci, i64, vp, vp]
     L.hyper_attn_levels.argtypes = [i64, ci, i64, ctypes.POINTER(ci), ctypes.POINTER(i64)]
     L.hyper_attn_debug_copy.argtypes = [vp, ci, ci, vp, ctypes.c_size_t]
@@ -165,6 +166,12 @@ class HyperAttention:
     def exact(self, Q, K, V, O, *, n, d, heads, causal):
         """Exact softmax attention (device tensors) on the tensor-core kernel; enqueued on the handle's stream."""
         self._check(lib().hyper_attn_exact(self._h, _ptr(Q), _ptr(K), _ptr(V), _ptr(O), n, d, heads, int(causal)))
+
+    def backward(self, Q, K, V, dO, dQ, dK, dV, *, n, d, heads, block, m, r, causal, seed):
+        """Gradients of sum(dO * O) into fp32 device tensors dQ, dK, dV (the forward is recomputed); enqueued on
+        the handle's stream."""
+        self._check(lib().hyper_attn_backward(self._h, _ptr(Q), _ptr(K), _ptr(V), _ptr(dO), _ptr(dQ), _ptr(dK),
+                                              _ptr(dV), n, d, heads, block, m, r, int(causal), seed))
 
     def diagnostics(self, Q, K, *, n, d, heads, block, r, seed, first_col=0):
         """(alpha, kappa) arrays of length batch*heads for device tensors Q, K (synchronous)."""

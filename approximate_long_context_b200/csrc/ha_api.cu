@@ -41,6 +41,8 @@ struct hyper_attn_s {
         size_t rn_nrm, rn_csum, rn_cdf, rn_S, rn_lw, rn_bytes;
     } lay{};
     bool have_last = false;
+    // the forward pass runs for a backward pass: fp32 O, per-row log normalisers captured (causal: final ones)
+    bool bwd = false;
     int last_launches = 0;
     int last_kernel = 0;
     // profiling: event pairs recorded around kernel-class launches
@@ -314,8 +316,9 @@ int run_forward(hyper_attn_t h, const void *Q, const void *K, const void *V, voi
                 uint64_t seed, int64_t bh_offset, bool sort_only = false) {
     cudaStream_t st = static_cast<cudaStream_t>(h->opt.stream);
     const int dtype = h->opt.dtype;
-    const int out_dtype = h->opt.out_dtype < 0 ? dtype : h->opt.out_dtype;
+    const int out_dtype = h->bwd ? HA_DTYPE_FP32 : (h->opt.out_dtype < 0 ? dtype : h->opt.out_dtype);
     const int esz = dtype == HA_DTYPE_BF16 ? 2 : 4;
+    const int capture = h->opt.debug_captures || h->bwd;
     bool use_tc = false;
     if (h->opt.kernel == HA_KERNEL_TC) {
         if (dtype != HA_DTYPE_BF16) return fail(h, HA_ERR_UNSUPPORTED, "tensor-core kernels need bf16 inputs");
@@ -326,7 +329,7 @@ int run_forward(hyper_attn_t h, const void *Q, const void *K, const void *V, voi
 
     const bool rownorm = h->opt.sampling == HA_SAMPLING_ROWNORM && s.m > 0 && !sort_only;
     hyper_attn_s::Layout lay;
-    const size_t bytes = plan_layout(s, esz, h->opt.debug_captures, rownorm, &lay);
+    const size_t bytes = plan_layout(s, esz, capture, rownorm, &lay);
     int rc = ensure_workspace(h, bytes);
     if (rc) return rc;
     // a layout change invalidates resident draws only if their offsets moved
@@ -343,7 +346,7 @@ int run_forward(hyper_attn_t h, const void *Q, const void *K, const void *V, voi
     uint8_t *near = ws + lay.near;
     int32_t *hist = reinterpret_cast<int32_t *>(ws + lay.hist);
     int32_t *perm_tmp = reinterpret_cast<int32_t *>(ws + lay.perm_tmp);
-    float *lse = h->opt.debug_captures ? reinterpret_cast<float *>(ws + lay.lse) : nullptr;
+    float *lse = capture ? reinterpret_cast<float *>(ws + lay.lse) : nullptr;
     float *Opart = reinterpret_cast<float *>(ws + lay.Opart);
     float *Lpart = reinterpret_cast<float *>(ws + lay.Lpart);
     int *status = reinterpret_cast<int *>(ws + lay.status);
@@ -444,12 +447,15 @@ int run_forward(hyper_attn_t h, const void *Q, const void *K, const void *V, voi
         int k = -2;
         ev = prof_begin();
         if (use_tc && family != HA_KERNEL_SIMT) family = HA_KERNEL_TC;
-        if (use_tc) k = ha::launch_causal_base_tc(Q, K, V, s.bh, s.n, s.d, s.leaf, s.levels, Opart, Lpart, O, out_dtype,
-                                                  status, st, stall_ns);
-        if (k == -2 && h->opt.kernel != HA_KERNEL_TC) family = HA_KERNEL_SIMT;
-        if (k == -2 && h->opt.kernel != HA_KERNEL_TC)
+        // a backward pass needs each row's final log normaliser, which the SIMT kernel writes
+        if (use_tc && !h->bwd)
+            k = ha::launch_causal_base_tc(Q, K, V, s.bh, s.n, s.d, s.leaf, s.levels, Opart, Lpart, O, out_dtype, status,
+                                          st, stall_ns);
+        const bool simt_ok = h->opt.kernel != HA_KERNEL_TC || h->bwd;
+        if (k == -2 && simt_ok) family = HA_KERNEL_SIMT;
+        if (k == -2 && simt_ok)
             k = ha::launch_causal_base_simt(Q, K, V, dtype, s.bh, s.n, s.d, s.leaf, s.levels, Opart, Lpart, O,
-                                            out_dtype, st);
+                                            out_dtype, st, h->bwd ? lse : nullptr);
         prof_end(ev, HA_KC_CAUSAL_BASE, k);
         if ((rc = count(k, "causal base"))) return rc;
     }
@@ -552,6 +558,74 @@ int hyper_attn_forward(hyper_attn_t h, const void *Q, const void *K, const void 
     if (rc) return rc;
     DeviceGuard g(h->device);
     return run_forward(h, Q, K, V, O, s, seed, h->opt.bh_offset);
+}
+
+int hyper_attn_backward(hyper_attn_t h, const void *Q, const void *K, const void *V, const void *dO, float *dQ,
+                        float *dK, float *dV, int64_t n, int d, int heads, int block, int m, int r, int causal,
+                        uint64_t seed) {
+    if (!h) return HA_ERR_INVALID_ARG;
+    h->err.clear();
+    if (!Q || !K || !V || !dO || !dQ || !dK || !dV) return fail(h, HA_ERR_INVALID_ARG, "null tensor pointer");
+    const void *all[7] = {Q, K, V, dO, dQ, dK, dV};
+    for (const void *p : all)
+        if (!aligned16(p)) return fail(h, HA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    for (int i = 4; i < 7; ++i)
+        for (int j = 0; j < 7; ++j)
+            if (i != j && all[i] == all[j]) return fail(h, HA_ERR_INVALID_ARG, "gradients must not alias any tensor");
+    if (heads <= 0) return fail(h, HA_ERR_INVALID_ARG, "heads must be positive");
+    Shape s{};
+    int rc = check_shape(h, n, d, h->opt.batch * heads, block, m, r, causal, &s);
+    if (rc) return rc;
+    DeviceGuard g(h->device);
+    cudaStream_t st = static_cast<cudaStream_t>(h->opt.stream);
+    const int dtype = h->opt.dtype;
+    const int esz = dtype == HA_DTYPE_BF16 ? 2 : 4;
+    const bool rownorm = h->opt.sampling == HA_SAMPLING_ROWNORM && s.m > 0;
+    // workspace: the forward's layout (with the captured log normalisers), then O (fp32) and g = dO . O
+    hyper_attn_s::Layout lay;
+    const size_t fwd = align_up(plan_layout(s, esz, 1, rownorm, &lay));
+    const size_t rows = static_cast<size_t>(s.bh) * static_cast<size_t>(s.n);
+    const size_t obytes = align_up(sizeof(float) * rows * s.d);
+    rc = ensure_workspace(h, fwd + obytes + align_up(sizeof(float) * rows));
+    if (rc) return rc;
+    float *Of = reinterpret_cast<float *>(h->ws + fwd);
+    float *gq = reinterpret_cast<float *>(h->ws + fwd + obytes);
+    h->bwd = true;
+    rc = run_forward(h, Q, K, V, Of, s, seed, h->opt.bh_offset);
+    h->bwd = false;
+    if (rc) return rc;
+    int launches = h->last_launches;
+    auto count = [&](int k, const char *what) -> int {
+        if (k < 0) return fail(h, HA_ERR_CUDA, "%s launch failed: %s", what, cudaGetErrorString(cudaGetLastError()));
+        launches += k;
+        return HA_OK;
+    };
+    const size_t gbytes = sizeof(float) * rows * s.d;
+    HA_CUDA(h, cudaMemsetAsync(dQ, 0, gbytes, st));
+    HA_CUDA(h, cudaMemsetAsync(dK, 0, gbytes, st));
+    HA_CUDA(h, cudaMemsetAsync(dV, 0, gbytes, st));
+    unsigned char *ws = h->ws;
+    const float *L = reinterpret_cast<const float *>(ws + h->lay.lse);
+    if ((rc = count(ha::launch_bwd_rowdot(dO, dtype, Of, static_cast<int64_t>(rows), s.d, gq, st), "backward dot")))
+        return rc;
+    const int32_t *S = reinterpret_cast<const int32_t *>(ws + h->lay.S);
+    const int32_t *Srn = rownorm ? reinterpret_cast<const int32_t *>(ws + h->lay.rn_S) : nullptr;
+    const float *lwrn = rownorm ? reinterpret_cast<const float *>(ws + h->lay.rn_lw) : nullptr;
+    for (int i = 0; (!s.causal || s.levels > 0) && i < s.nlev; ++i) {
+        const ha::Level lv = make_level(s, s.causal ? i + 1 : 0);
+        const int32_t *perm = reinterpret_cast<const int32_t *>(ws + h->lay.perm[i]);
+        const int32_t *inv = reinterpret_cast<const int32_t *>(ws + h->lay.inv[i]);
+        rc = count(ha::launch_bwd_level(lv, Q, K, V, dO, dtype, s.d, perm, inv, S, s.m, s.nodes_total, Srn, lwrn, L,
+                                        gq, dQ, dK, dV, st),
+                   "backward level");
+        if (rc) return rc;
+    }
+    if (s.causal &&
+        (rc = count(ha::launch_bwd_leaf(Q, K, V, dO, dtype, s.bh, s.n, s.d, s.leaf, L, gq, dQ, dK, dV, st),
+                    "backward leaves")))
+        return rc;
+    h->last_launches = launches;
+    return HA_OK;
 }
 
 int hyper_attn_diagnostics(hyper_attn_t h, const void *Q, const void *K, int64_t n, int d, int heads, int block,

@@ -152,7 +152,7 @@ template <int D>
 __global__ void __launch_bounds__(kWarpsPerCta * 32) causal_base_simt_kernel(
     const void *__restrict__ Q, const void *__restrict__ K, const void *__restrict__ V, int dtype, int64_t bh,
     int64_t n, int64_t leaf, int levels, const float *__restrict__ Opart, const float *__restrict__ Lpart,
-    void *__restrict__ O, int out_dtype) {
+    void *__restrict__ O, int out_dtype, float *__restrict__ Lout) {
     constexpr int DPL = D / 32;
     const int lane = threadIdx.x & 31;
     const int64_t wg = static_cast<int64_t>(blockIdx.x) * kWarpsPerCta + (threadIdx.x >> 5);
@@ -196,6 +196,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) causal_base_simt_kernel(
     }
 #pragma unroll
     for (int c = 0; c < DPL; ++c) store_out(O, head + qrow * D + col + c, Ocur[c], out_dtype);
+    if (Lout && lane == 0) Lout[wg] = Lcur;   // the row's final log normaliser (for the backward pass)
 }
 
 }  // namespace
@@ -219,14 +220,14 @@ int launch_attn_simt(const Level &lv, const void *Q, const void *K, const void *
 
 int launch_causal_base_simt(const void *Q, const void *K, const void *V, int dtype, int64_t bh, int64_t n, int d,
                             int64_t leaf, int levels, const float *Opart, const float *Lpart, void *O,
-                            int out_dtype, cudaStream_t st) {
+                            int out_dtype, cudaStream_t st, float *Lout) {
     const int64_t grid = (bh * n + kWarpsPerCta - 1) / kWarpsPerCta;
     if (d == 64)
         causal_base_simt_kernel<64><<<static_cast<unsigned>(grid), kWarpsPerCta * 32, 0, st>>>(
-            Q, K, V, dtype, bh, n, leaf, levels, Opart, Lpart, O, out_dtype);
+            Q, K, V, dtype, bh, n, leaf, levels, Opart, Lpart, O, out_dtype, Lout);
     else if (d == 128)
         causal_base_simt_kernel<128><<<static_cast<unsigned>(grid), kWarpsPerCta * 32, 0, st>>>(
-            Q, K, V, dtype, bh, n, leaf, levels, Opart, Lpart, O, out_dtype);
+            Q, K, V, dtype, bh, n, leaf, levels, Opart, Lpart, O, out_dtype, Lout);
     else
         return -1;
     return cudaPeekAtLastError() == cudaSuccess ? 1 : -1;

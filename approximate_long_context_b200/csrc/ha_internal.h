@@ -58,9 +58,10 @@ int launch_attn_simt(const Level &lv, const void *Q, const void *K, const void *
                      const int32_t *Srn = nullptr, const float *lwrn = nullptr);
 
 // SIMT exact causal attention on leaves of `leaf` rows, merged with the parts of levels 1..L.
+// Lout (optional): the final log normaliser of every row [bh][n].
 int launch_causal_base_simt(const void *Q, const void *K, const void *V, int dtype, int64_t bh, int64_t n,
                             int d, int64_t leaf, int levels, const float *Opart, const float *Lpart,
-                            void *O, int out_dtype, cudaStream_t st);
+                            void *O, int out_dtype, cudaStream_t st, float *Lout = nullptr);
 
 // Tensor-core (tcgen05) kernels; return -2 when a shape is not supported by the tensor-core path.
 int launch_attn_tc(const Level &lv, const void *Q, const void *K, const void *V, int d,
@@ -101,6 +102,17 @@ RowNormGeom rownorm_geometry(int64_t n, int causal, int levels, int m, int64_t n
 int launch_rownorm_draws(const RowNormGeom &g, const void *V, int dtype, int d, int64_t bh, uint64_t seed,
                          int64_t bh_offset, float *nrm, double *csum, double *cdf, int32_t *S, float *logw,
                          cudaStream_t st);
+
+// Backward pass (ha_backward.cu): g[rows] = dO . O (O fp32); the key terms of one level and of the exact causal
+// leaves, adding into fp32 dQ, dK, dV [bh][n][d] (zeroed by the caller). L: final log normaliser [bh][n].
+int launch_bwd_rowdot(const void *dO, int dtype, const float *O, int64_t rows, int d, float *g, cudaStream_t st);
+int launch_bwd_level(const Level &lv, const void *Q, const void *K, const void *V, const void *dO, int dtype, int d,
+                     const int32_t *perm, const int32_t *inv, const int32_t *S, int m, int64_t nodes_total,
+                     const int32_t *Srn, const float *lwrn, const float *L, const float *g, float *dQ, float *dK,
+                     float *dV, cudaStream_t st);
+int launch_bwd_leaf(const void *Q, const void *K, const void *V, const void *dO, int dtype, int64_t bh, int64_t n,
+                    int d, int64_t leaf, const float *L, const float *g, float *dQ, float *dK, float *dV,
+                    cudaStream_t st);
 
 // ---- host-side draws (ha_draws.cpp) ----
 void draw_projection(uint64_t seed, int d, int r, float *P);

@@ -376,6 +376,28 @@ def run_ours(args, w: wl.Workload):
         diag = {"rows": nd, "head": 0, "alpha": float(a0[0]), "alpha_without_first_32": float(a32[0]),
                 "kappa": float(k0[0]), "ms": g0.elapsed_time(g1)}
 
+    # optional: the backward pass (gradients of sum(dO * O); recomputes the forward) on the same inputs
+    bwd = None
+    if args.backward:
+        gen = torch.Generator(device=dev).manual_seed(5)
+        dO = torch.randn(Q.shape, generator=gen, device=dev, dtype=torch.float32).to(Q.dtype)
+        grads = [torch.empty(Q.shape, dtype=torch.float32, device=dev) for _ in range(3)]
+        ha.set_options(dtype=w.dtype, batch=w.batch, causal_base=w.base or 4096, stream=stream.cuda_stream,
+                       kernel=args.kernel, bh_offset=sh.offset, sampling=args.sampling)
+        ha.backward(Q, K, V, dO, *grads, **kw)   # warm-up
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        b0.record(stream)
+        for _ in range(args.backward):
+            ha.backward(Q, K, V, dO, *grads, **kw)
+        b1.record(stream)
+        torch.cuda.synchronize(dev)
+        assert ha.status() == 0, ha.last_error()
+        bms = max_over_ranks(b0.elapsed_time(b1) / args.backward, dev)
+        bwd = {"ms_per_step": bms, "value": units / (bms * 1e-3) / 1e6, "unit": UNIT, "steps": args.backward,
+               "kernels": "forward recompute, then SIMT fp32 gradient kernels (dK, dV by atomic adds)"}
+        del dO, grads
+
     # roofline of the dominant kernel class; sort and attention launch once per level
     peaks, peak_src = load_peaks()
     family = ha.last_kernel()
@@ -440,6 +462,8 @@ def run_ours(args, w: wl.Workload):
         }
         if diag is not None:
             line["diagnostics"] = diag
+        if bwd is not None:
+            line["backward"] = bwd
         print(json.dumps(line), flush=True)
     ha.close()
     if world > 1:
@@ -461,6 +485,8 @@ def main():
                     help="run the workload with this many heads instead of its own (small profiler captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-exact", action="store_true", help="skip the same-box exact-attention comparison")
+    ap.add_argument("--backward", type=int, default=0, metavar="STEPS",
+                    help="also time the backward pass over this many steps (after one warm-up)")
     ap.add_argument("--diagnostics", action="store_true",
                     help="also report the hardness diagnostics (alpha, kappa) of the first 4096 rows of head 0")
     args = ap.parse_args()

@@ -131,6 +131,25 @@ HA_API int hyper_attn_exact(hyper_attn_t h, const void *Q, const void *K, const 
                             int64_t n, int d, int heads, int causal);
 
 /*
+ * Backward pass: the gradients of sum(dO * O) with respect to Q, K and V, where O is the forward estimate of
+ * hyper_attn_forward with the same arguments and options (the sort permutations and the sample draws are
+ * held fixed: they are constants of the forward pass). Every row's estimate is a weighted softmax over a
+ * sparse key set (its sortLSH block or causal leaf with weight 1, uniform samples outside the block with N/m,
+ * row-norm draws with 1/(m p_j) in the numerator only), so ("HyperAttention: Long-context Attention in
+ * Near-Linear Time", research-map summary, "Key results": the speed-ups are for forward and backward):
+ *   dS_qk = Wn e^{s_qk - L_q} (dO_q . v_k) - Wd e^{s_qk - L_q} (dO_q . O_q),
+ *   dQ = dS K, dK = dS^T Q, dV_k = sum_q Wn e^{s_qk - L_q} dO_q.
+ *   Q, K, V, dO  device pointers, [batch, heads, n, d] of the options' dtype (read only).
+ *   dQ, dK, dV   device pointers, [batch, heads, n, d] fp32, written (overwritten); no aliasing.
+ * The forward pass is recomputed (its O in fp32 and the log normalisers stay in the workspace); the gradients
+ * are accumulated by SIMT fp32 kernels, dK and dV with atomic adds, so the last bits may vary between runs.
+ * Enqueued on the options' stream; same argument checks and error codes as hyper_attn_forward.
+ */
+HA_API int hyper_attn_backward(hyper_attn_t h, const void *Q, const void *K, const void *V, const void *dO, float *dQ,
+                               float *dK, float *dV, int64_t n, int d, int heads, int block, int m, int r, int causal,
+                               uint64_t seed);
+
+/*
  * Hardness diagnostics of the attention matrices of small non-causal problems ("HyperAttention: Long-context
  * Attention in Near-Linear Time", research-map summary, "Approach" and "Key results", abstract page: the
  * guarantee rests on the max column norm of the normalised attention matrix and on the ratio of row norms

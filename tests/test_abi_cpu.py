@@ -81,3 +81,27 @@ def test_levels(lib):
         binding.levels(3 * 4096, True, 4096)
     with pytest.raises(binding.HAError):
         binding.draw(1, 64, 4, 1, 100, 101, causal=False)
+
+
+def test_options_struct_mirrors_the_header(tmp_path):
+    """The binding's ctypes Options has the C struct's size and field offsets (compiled here with gcc)."""
+    fields = [f for f, _ in binding.Options._fields_]
+    src = tmp_path / "layout.c"
+    body = "".join(f'    printf("{f} %zu\\n", offsetof(ha_options, {f}));\n' for f in fields)
+    src.write_text('#include <stddef.h>\n#include <stdio.h>\n#include "hyper_attn.h"\nint main(void) {\n'
+                   '    printf("size %zu\\n", sizeof(ha_options));\n' + body + "    return 0;\n}\n")
+    exe = tmp_path / "layout"
+    import subprocess
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    out = dict(line.split() for line in subprocess.run([str(exe)], capture_output=True, text=True,
+                                                       check=True).stdout.splitlines())
+    assert int(out["size"]) == ctypes.sizeof(binding.Options)
+    for f in fields:
+        assert int(out[f]) == getattr(binding.Options, f).offset, f
+
+
+def test_default_options_match_the_binding_defaults(lib):
+    o = binding.Options()
+    lib.hyper_attn_default_options(ctypes.byref(o))
+    assert (o.dtype, o.out_dtype, o.batch, o.causal_base, o.kernel, o.debug_captures, o.bh_offset,
+            o.test_stall_ms, o.sampling) == (0, -1, 1, 4096, 0, 0, 0, 0, 0)

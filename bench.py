@@ -63,6 +63,11 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
+def nlev_of(w: wl.Workload) -> int:
+    """Causal levels of a workload (0 for non-causal)."""
+    return int(round(np.log2(w.n // w.base))) if (w.causal and w.n > w.base) else 0
+
+
 def algorithmic(w: wl.Workload, cls: str, sampling: str = "uniform"):
     """Algorithmic work per launch of a kernel class: (bytes, flops)."""
     e = 2 if w.dtype == "bf16" else 4
@@ -394,8 +399,19 @@ def run_ours(args, w: wl.Workload):
         torch.cuda.synchronize(dev)
         assert ha.status() == 0, ha.last_error()
         bms = max_over_ranks(b0.elapsed_time(b1) / args.backward, dev)
+        # algorithmic FLOPs of the gradient kernels: per (query, key) term the score, dO.v, and the dQ, dK, dV
+        # updates, 2d each; terms per query as in the forward (uniform samples count once with row-norm
+        # sampling plus the draws), plus the exact causal leaves (c/2 keys per query on average)
+        terms = w.bh * (w.n if not w.causal else (w.n // 2) * nlev_of(w)) * (
+            min(w.block, w.n if not w.causal else w.n // 2) + w.m * (2 if args.sampling == "rownorm" else 1))
+        if w.causal:
+            terms += w.bh * w.n * min(w.base, w.n) / 2
+        bflops = 10.0 * w.d * terms
         bwd = {"ms_per_step": bms, "value": units / (bms * 1e-3) / 1e6, "unit": UNIT, "steps": args.backward,
-               "kernels": "forward recompute, then SIMT fp32 gradient kernels (dK, dV by atomic adds)"}
+               "kernels": "forward recompute, then SIMT fp32 gradient kernels (dK, dV by atomic adds)",
+               "roofline": {"bound": "alu", "achieved": bflops / (bms * 1e-3) / 1e12, "peak": FP32_SIMT_PEAK_TFLOPS,
+                            "unit": "TFLOP/s", "frac": bflops / (bms * 1e-3) / 1e12 / FP32_SIMT_PEAK_TFLOPS,
+                            "note": "whole backward call (forward recompute included) against the FP32 ALU peak"}}
         del dO, grads
 
     # roofline of the dominant kernel class; sort and attention launch once per level

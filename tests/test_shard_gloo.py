@@ -113,3 +113,19 @@ def test_problem_index_keys_the_draws(ora):
         a = _run_problem(Q[0], K[0], V[0], 3, ora, sampling)
         b = _run_problem(Q[0], K[0], V[0], 0, ora, sampling)
         assert not np.array_equal(a, b)
+
+
+def test_backward_shards_by_problem(ora):
+    """The backward pass of a problem depends only on its own inputs and global index: per-rank slices of the
+    job's gradients equal the whole job's (each rank runs the problems of its range with their global index)."""
+    Q, K, V = wl.make_inputs(N, D, G, data_seed=DATA_SEED, dtype="fp32")
+    dO = np.random.default_rng(4).standard_normal((G, N, D)).astype(np.float32)
+    kw = dict(block=64, m=32, r=6, causal=False, seed=77)
+    whole = [ora.backward(Q[g], K[g], V[g], dO[g], bh=g, **kw)["dK"] for g in range(G)]
+    for world in (2, 3):
+        for rank in range(world):
+            s = shard.shard_problems(G, world, rank)
+            for i, g in enumerate(range(s.offset, s.offset + s.count)):
+                Qs, Ks, Vs = wl.make_inputs(N, D, G, data_seed=DATA_SEED, dtype="fp32", heads=[g])
+                got = ora.backward(Qs[0], Ks[0], Vs[0], dO[g], bh=g, **kw)["dK"]
+                assert np.array_equal(got, whole[g])

@@ -82,6 +82,10 @@ def _load():
                                  ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_uint64,
                                  ctypes.c_int64, ctypes.c_int, _f64p, _f64p, _f64p, _f64p, _f64p]
     lib.ora_backward.restype = ctypes.c_int
+    lib.ora_backward_rows.argtypes = [_f32p, _f32p, _f32p, _f32p, ctypes.c_int64, ctypes.c_int, ctypes.c_int64,
+                                      ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_uint64,
+                                      ctypes.c_int64, ctypes.c_int, vp, ctypes.c_int64, _f64p]
+    lib.ora_backward_rows.restype = ctypes.c_int
     lib.ora_num_threads.argtypes = []
     lib.ora_num_threads.restype = ctypes.c_int
     _lib = lib
@@ -237,6 +241,21 @@ def backward(Q, K, V, dO, *, block: int, m: int, r: int, causal: bool, seed: int
     _check(_load().ora_backward(Q, K, V, dO, n, d, block, m, r, int(causal), base, seed, bh, SAMPLING[sampling],
                                 out["dQ"], out["dK"], out["dV"], out["O"], out["L"]), "backward")
     return out
+
+
+def backward_rows(Q, K, V, dO, rows, *, block: int, m: int, r: int, causal: bool, seed: int, bh: int = 0,
+                  base: int = 0, sampling: str = "uniform") -> np.ndarray:
+    """dQ (len(rows), d) float64 of the selected rows, for any n (no dense weights; see oracle.c)."""
+    Q = np.ascontiguousarray(Q, np.float32)
+    K = np.ascontiguousarray(K, np.float32)
+    V = np.ascontiguousarray(V, np.float32)
+    dO = np.ascontiguousarray(dO, np.float32)
+    n, d = Q.shape
+    sel = np.ascontiguousarray(rows, np.int64)
+    dQ = np.zeros((max(len(sel), 1), d), np.float64)
+    _check(_load().ora_backward_rows(Q, K, V, dO, n, d, block, m, r, int(causal), base, seed, bh, SAMPLING[sampling],
+                                     _ptr(sel), len(sel), dQ), "backward_rows")
+    return dQ[:len(sel)]
 
 
 def exact_attention(Q, K, V, *, causal: bool, rows=None) -> np.ndarray:

@@ -853,6 +853,127 @@ int ora_backward(const float *Q, const float *K, const float *V, const float *dO
     return rc;
 }
 
+/*
+ * dQ of selected rows only, for problems too large for the dense weights: the same key terms and formula as
+ * ora_backward (dS_qk = e^{s_qk - L_q} (Wn (dO_q . v_k) - Wd (dO_q . O_q)), dQ_q = sum_k dS_qk k_k), visited
+ * per subproblem like ora_forward_sampling. O_q and L_q come from ora_forward_sampling for the same rows.
+ */
+static int sub_dq(const float *Qr, const float *Kr, const float *Vr, const float *dOr, int64_t N, int d,
+                  const uint16_t *rq, const uint16_t *rk, int64_t block, const int32_t *S, int m, const int32_t *Srn,
+                  const double *lwrn, const int64_t *lq, const int64_t *ts, int64_t cnt, const double *L,
+                  const double *g, double *dQ)
+{
+    int64_t bp = block < N ? block : N;
+    if (bp <= 0 || N % bp != 0) return ORA_EINVAL;
+    int32_t *permQ = (int32_t *)malloc(sizeof(int32_t) * (size_t)N);
+    int32_t *permK = (int32_t *)malloc(sizeof(int32_t) * (size_t)N);
+    int64_t *posQ = (int64_t *)malloc(sizeof(int64_t) * (size_t)N);
+    int64_t *posK = (int64_t *)malloc(sizeof(int64_t) * (size_t)N);
+    int rc = (!permQ || !permK || !posQ || !posK) ? ORA_ENOMEM : ORA_OK;
+    if (rc == ORA_OK) rc = ora_sort_segment(rq, N, permQ);
+    if (rc == ORA_OK) rc = ora_sort_segment(rk, N, permK);
+    if (rc == ORA_OK) {
+        for (int64_t p = 0; p < N; ++p) { posQ[permQ[p]] = p; posK[permK[p]] = p; }
+        const double lw = m > 0 ? log((double)N / (double)m) : 0.0;
+        for (int64_t c = 0; c < cnt; ++c) {
+            const int64_t q = lq[c], t = ts[c], i = posQ[q] / bp;
+            const float *qv = Qr + q * d, *go = dOr + q * d;
+            double *dq = dQ + t * d;
+            /* one term: key k with log weights (ln_wn, ln_wd); -INFINITY = weight 0 */
+#define ORA_TERM(kk, ln_wn, ln_wd)                                                                            \
+            do {                                                                                              \
+                const int64_t k_ = (kk);                                                                      \
+                const double s_ = dot_fd(qv, Kr + k_ * d, d);                                                 \
+                const double en_ = (ln_wn) == -INFINITY ? 0.0 : exp(s_ + (ln_wn) - L[t]);                     \
+                const double ed_ = (ln_wd) == -INFINITY ? 0.0 : exp(s_ + (ln_wd) - L[t]);                     \
+                const double dov_ = dot_fd(go, Vr + k_ * d, d);                                               \
+                const double ds_ = en_ * dov_ - ed_ * g[t];                                                   \
+                for (int x = 0; x < d; ++x) dq[x] += ds_ * (double)Kr[k_ * d + x];                            \
+            } while (0)
+            for (int64_t j = 0; j < bp; ++j) ORA_TERM(permK[i * bp + j], 0.0, 0.0);
+            for (int u = 0; u < m; ++u) {
+                if (posK[S[u]] / bp == i) continue;
+                ORA_TERM(S[u], Srn ? -INFINITY : lw, lw);
+            }
+            for (int u = 0; Srn && u < m; ++u) {
+                if (Srn[u] < 0 || posK[Srn[u]] / bp == i) continue;
+                ORA_TERM(Srn[u], lwrn[u], -INFINITY);
+            }
+#undef ORA_TERM
+        }
+    }
+    free(permQ); free(permK); free(posQ); free(posK);
+    return rc;
+}
+
+int ora_backward_rows(const float *Q, const float *K, const float *V, const float *dO, int64_t n, int d,
+                      int64_t block, int m, int r, int causal, int64_t base, uint64_t seed, int64_t bh, int sampling,
+                      const int64_t *rows, int64_t nrows, double *dQ)
+{
+    if (nrows <= 0) return ORA_EINVAL;
+    int rc = ORA_OK;
+    double *O = (double *)malloc(sizeof(double) * (size_t)(nrows * d));
+    double *L = (double *)malloc(sizeof(double) * (size_t)nrows);
+    double *g = (double *)malloc(sizeof(double) * (size_t)nrows);
+    float *P = (float *)malloc(sizeof(float) * (size_t)(d * (r > 0 ? r : 1)));
+    uint16_t *rank = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)(2 * n));
+    uint8_t *near = (uint8_t *)malloc((size_t)(2 * n));
+    int32_t *S = (int32_t *)malloc(sizeof(int32_t) * (size_t)(m > 0 ? m : 1));
+    int32_t *Srn = (int32_t *)malloc(sizeof(int32_t) * (size_t)(m > 0 ? m : 1));
+    double *lw = (double *)malloc(sizeof(double) * (size_t)(m > 0 ? m : 1));
+    int64_t *lq = (int64_t *)malloc(sizeof(int64_t) * (size_t)nrows);
+    int64_t *ts = (int64_t *)malloc(sizeof(int64_t) * (size_t)nrows);
+    if (!O || !L || !g || !P || !rank || !near || !S || !Srn || !lw || !lq || !ts) { rc = ORA_ENOMEM; goto out; }
+    rc = ora_forward_sampling(Q, K, V, n, d, block, m, r, causal, base, seed, bh, rows, nrows, O, L, NULL, NULL,
+                              rank, near, sampling);
+    if (rc != ORA_OK) goto out;
+    for (int64_t t = 0; t < nrows; ++t) {
+        g[t] = 0.0;
+        for (int x = 0; x < d; ++x) g[t] += (double)dO[rows[t] * d + x] * O[t * d + x];
+    }
+    memset(dQ, 0, sizeof(double) * (size_t)(nrows * d));
+    if (!causal) {
+        rc = ora_draw_samples(seed, bh, 1, n, m, S);
+        if (rc == ORA_OK && sampling) rc = ora_draw_rownorm(seed, bh, 1, V, n, d, m, Srn, lw);
+        for (int64_t t = 0; t < nrows; ++t) { lq[t] = rows[t]; ts[t] = t; }
+        if (rc == ORA_OK)
+            rc = sub_dq(Q, K, V, dO, n, d, rank, rank + n, block, S, m, sampling ? Srn : NULL, lw, lq, ts, nrows, L,
+                        g, dQ);
+        goto out;
+    }
+    {
+        const int64_t leaf = base < n ? base : n;
+        for (int64_t t = 0; t < nrows; ++t) {   /* exact causal leaf: keys q - q % leaf .. q, weight 1 */
+            const int64_t q = rows[t];
+            for (int64_t k = q - q % leaf; k <= q; ++k) {
+                const double s_ = dot_fd(Q + q * d, K + k * d, d);
+                const double e_ = exp(s_ - L[t]);
+                const double ds_ = e_ * (dot_fd(dO + q * d, V + k * d, d) - g[t]);
+                for (int x = 0; x < d; ++x) dQ[t * d + x] += ds_ * (double)K[k * d + x];
+            }
+        }
+        for (int64_t len = n; len > leaf && rc == ORA_OK; len >>= 1) {
+            const int64_t half = len / 2, nodes = n / len;
+            for (int64_t j = 0; j < nodes && rc == ORA_OK; ++j) {
+                const int64_t s0 = j * len, node = nodes + j;
+                int64_t cnt = 0;
+                for (int64_t t = 0; t < nrows; ++t)
+                    if (rows[t] >= s0 + half && rows[t] < s0 + len) { lq[cnt] = rows[t] - (s0 + half); ts[cnt] = t; ++cnt; }
+                if (cnt == 0) continue;
+                rc = ora_draw_samples(seed, bh, node, half, m, S);
+                if (rc == ORA_OK && sampling) rc = ora_draw_rownorm(seed, bh, node, V + s0 * d, half, d, m, Srn, lw);
+                if (rc == ORA_OK)
+                    rc = sub_dq(Q + (s0 + half) * d, K + s0 * d, V + s0 * d, dO + (s0 + half) * d, half, d,
+                                rank + s0 + half, rank + n + s0, block, S, m, sampling ? Srn : NULL, lw, lq, ts, cnt,
+                                L, g, dQ);
+            }
+        }
+    }
+out:
+    free(O); free(L); free(g); free(P); free(rank); free(near); free(S); free(Srn); free(lw); free(lq); free(ts);
+    return rc;
+}
+
 int ora_num_threads(void)
 {
 #ifdef _OPENMP

@@ -629,3 +629,17 @@ def test_backward_identities(ora, causal, sampling):
     lhs = float((out["dV"] * V.astype(np.float64)).sum())
     rhs = float((out["O"] * dO.astype(np.float64)).sum())
     assert lhs == pytest.approx(rhs, rel=1e-12, abs=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("sampling", ["uniform", "rownorm"])
+def test_backward_rows_equal_dense(ora, causal, sampling):
+    """dQ of selected rows, computed per subproblem without dense weights (for large n), equals the dense
+    backward's rows."""
+    n, d = 512, 16
+    Q, K, V = rand_qkv(n, d, 65)
+    dO = np.random.default_rng(10).standard_normal((n, d)).astype(np.float32)
+    rows = np.array([0, 1, 63, 64, 200, 255, 256, 300, 511])
+    kw = dict(block=32, m=24, r=5, causal=causal, base=64, seed=6, bh=3, sampling=sampling)
+    dense = ora.backward(Q, K, V, dO, **kw)["dQ"][rows]
+    np.testing.assert_allclose(ora.backward_rows(Q, K, V, dO, rows, **kw), dense, rtol=1e-10, atol=1e-12)

@@ -4,11 +4,14 @@
 // up front and forbids allocation while it enqueues work, or a latency-critical loop that cannot afford
 // the device-wide synchronisation an allocation may cause. hyper_attn_forward_noalloc serves them: the
 // caller passes Q, K, V and O, and every scratch buffer of the pass (draws, ranks, flags, permutations,
-// sort histograms, status word) lives in one file-scope __device__ array of kNoAllocScratchBytes that each
-// GPU loading this library holds until the process exits. Calls share that array, so calls that overlap
-// on the GPU (on different streams, or from different host threads on different streams) race; callers
-// must order them. Host-side draws use file-scope host arrays under a mutex, so concurrent host calls are
-// serialised.
+// sort histograms) lives in one file-scope __device__ array of kNoAllocScratchBytes that each GPU loading
+// this library holds until the process exits. Calls share that array, so calls that overlap on the GPU (on
+// different streams, or from different host threads on different streams) race; callers must order them.
+// Host-side draws use file-scope host arrays under a mutex, so concurrent host calls are serialised. The
+// draws reach the device through copies from those pageable host arrays, which only hold outside stream
+// capture (a captured copy would read the arrays when the graph is replayed, after later calls changed
+// them), so a call made while its stream is capturing is refused. No kernel on this path waits on anything
+// on the device, so the path has no status word to report.
 #include <mutex>
 
 #include "../../include/hyper_attn.h"
@@ -23,8 +26,7 @@ constexpr int kMaxRBits = ha::kMaxPassBits;   // one counting-sort pass
 constexpr int kMaxDevices = 64;
 
 constexpr size_t al(size_t x) { return (x + 255) / 256 * 256; }
-constexpr size_t kStatusOff = 0;
-constexpr size_t kPOff = kStatusOff + 256;
+constexpr size_t kPOff = 0;
 constexpr size_t kSOff = kPOff + al(sizeof(float) * ha::kMaxR * 128);
 constexpr size_t kRankOff = kSOff + al(sizeof(int32_t) * kMaxProblems * kMaxM);
 constexpr size_t kNearOff = kRankOff + al(sizeof(uint16_t) * 2 * kMaxRows);
@@ -51,6 +53,9 @@ extern "C" int hyper_attn_forward_noalloc(const void *Q, const void *K, const vo
                                           int heads, int block, int m, int r, uint64_t seed, int dtype,
                                           void *stream) {
     if (!Q || !K || !V || !O) return HA_ERR_INVALID_ARG;
+    // the hash and attention kernels read rows with 16-byte copies
+    for (const void *p : {static_cast<const void *>(Q), K, V, static_cast<const void *>(O)})
+        if (reinterpret_cast<uintptr_t>(p) & 15u) return HA_ERR_INVALID_ARG;
     if (O == Q || O == K || O == V) return HA_ERR_INVALID_ARG;
     if (dtype != HA_DTYPE_BF16 && dtype != HA_DTYPE_FP32) return HA_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return HA_ERR_UNSUPPORTED;
@@ -73,6 +78,12 @@ extern "C" int hyper_attn_forward_noalloc(const void *Q, const void *K, const vo
     }
     unsigned char *base = static_cast<unsigned char *>(g_scratch_dev[dev]);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cap) != cudaSuccess) {
+        cudaGetLastError();
+        return HA_ERR_CUDA;
+    }
+    if (cap != cudaStreamCaptureStatusNone) return HA_ERR_UNSUPPORTED;
 
     // host draws (same definitions as every other entry point)
     ha::draw_projection(seed, d, r, g_P);
@@ -80,8 +91,7 @@ extern "C" int hyper_attn_forward_noalloc(const void *Q, const void *K, const vo
         if (ha::draw_samples(seed, static_cast<uint64_t>(h), 1, n, m, g_S + static_cast<int64_t>(h) * m, g_floyd))
             return HA_ERR_INVALID_ARG;
     // pageable-host copies return once the source has been staged, so the host arrays are free again
-    if (cudaMemsetAsync(base + kStatusOff, 0, 256, st) != cudaSuccess ||
-        cudaMemcpyAsync(base + kPOff, g_P, sizeof(float) * d * (r ? r : 1), cudaMemcpyHostToDevice, st) != cudaSuccess ||
+    if (cudaMemcpyAsync(base + kPOff, g_P, sizeof(float) * d * (r ? r : 1), cudaMemcpyHostToDevice, st) != cudaSuccess ||
         (m > 0 && cudaMemcpyAsync(base + kSOff, g_S, sizeof(int32_t) * heads * m, cudaMemcpyHostToDevice, st) !=
                       cudaSuccess)) {
         cudaGetLastError();
@@ -99,10 +109,13 @@ extern "C" int hyper_attn_forward_noalloc(const void *Q, const void *K, const vo
     int32_t *inv = reinterpret_cast<int32_t *>(base + kInvOff);
     int32_t *hist = reinterpret_cast<int32_t *>(base + kHistOff);
 
-    if (ha::launch_hash(Q, K, dtype, heads, n, d, P, r, rank, near, st) < 0) return HA_ERR_CUDA;
+    // a failed launch leaves its error behind: take it, so that the caller's next check starts clean
     const ha::SortPass pass{0, 1 << r};
-    if (ha::launch_sort_pass(lv, rank, pass, nullptr, hist, perm, inv, st) < 0) return HA_ERR_CUDA;
-    if (ha::launch_attn_simt(lv, Q, K, V, dtype, d, perm, inv, S, m, 1, O, dtype, nullptr, nullptr, nullptr, st) < 0)
+    if (ha::launch_hash(Q, K, dtype, heads, n, d, P, r, rank, near, st) < 0 ||
+        ha::launch_sort_pass(lv, rank, pass, nullptr, hist, perm, inv, st) < 0 ||
+        ha::launch_attn_simt(lv, Q, K, V, dtype, d, perm, inv, S, m, 1, O, dtype, nullptr, nullptr, nullptr, st) < 0) {
+        cudaGetLastError();
         return HA_ERR_CUDA;
+    }
     return HA_OK;
 }

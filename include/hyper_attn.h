@@ -252,18 +252,22 @@ HA_API int hyper_attn_destroy(hyper_attn_t h);
  * callers that cannot call cudaMalloc: plugins inside engines that reserve all device memory up front and
  * forbid allocation while enqueueing, and latency-critical loops that cannot afford the synchronisation an
  * allocation may cause.
- *   Q, K, V, O  device pointers, [heads, n, d] of type `dtype` (HA_DTYPE_BF16 or HA_DTYPE_FP32); O has the
- *               same type; O must not alias Q, K or V. Other arguments as in hyper_attn_forward (causal = 0).
+ *   Q, K, V, O  device pointers, [heads, n, d] of type `dtype` (HA_DTYPE_BF16 or HA_DTYPE_FP32), each
+ *               16-byte aligned; O has the same type; O must not alias Q, K or V. Other arguments as in
+ *               hyper_attn_forward (causal = 0).
  *   stream      cudaStream_t to enqueue on (NULL = legacy default stream) on the CURRENT device.
  * Limits (HA_ERR_INVALID_ARG beyond them, checked on the host before anything is enqueued):
- *   heads * n <= 65536, heads <= 64, m <= 512 and m <= n, r <= 10, d in {64, 128}.
+ *   heads * n <= 65536, heads <= 64, m <= 512 and m <= n, r <= 10, d in {64, 128}, n a multiple of
+ *   min(block, n), pointers 16-byte aligned.
  * All scratch memory (2.5 MiB at most) is one file-scope __device__ array that every GPU loading this
  * library holds until the process exits; no cudaMalloc, cudaFree or other allocating call is made.
  * The first call on a device resolves that array's device address with cudaGetSymbolAddress (with the
- * device current); make that first call before any stream capture. Every call reuses the same array and
- * leaves its contents behind; calls that overlap on the GPU race with each other, so order them (for
- * example, one stream). Host threads are serialised by a lock. Attention uses the SIMT kernels.
- * Returns after enqueueing; HA_ERR_CUDA if a CUDA call fails.
+ * device current). Every call reuses the same array and leaves its contents behind; calls that overlap on
+ * the GPU race with each other, so order them (for example, one stream). Host threads are serialised by a
+ * lock. The draws are copied from pageable host arrays that the next call overwrites, so calls must not
+ * be made while the stream is capturing: such a call returns HA_ERR_UNSUPPORTED and enqueues nothing.
+ * Attention uses the SIMT kernels, which have no device-side waits (no status word to read).
+ * Returns after enqueueing; HA_ERR_CUDA if a CUDA call fails (the CUDA error is cleared before returning).
  */
 HA_API int hyper_attn_forward_noalloc(const void *Q, const void *K, const void *V, void *O, int64_t n, int d,
                                       int heads, int block, int m, int r, uint64_t seed, int dtype, void *stream);

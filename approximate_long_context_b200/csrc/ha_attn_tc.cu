@@ -51,128 +51,15 @@
 
 #include "ha_common.cuh"
 #include "ha_internal.h"
-#include "ha_sm100.cuh"
+#include "ha_attn_items.cuh"
 
 namespace ha {
 namespace {
 
 using namespace sm100;
+using namespace attn;
 
 constexpr int kThreads = 384;
-constexpr int kKC = 128;                // keys per chunk
-constexpr int kMaxLevels = 16;
-constexpr int kMaxSampleList = 1024;    // sampled columns per problem handled by the tensor-core path
-constexpr int kMaxSampleListRn = 256;   // the same with row-norm sampling (m uniform samples + m draws)
-constexpr int kMaxBlock = 1024;         // rows per sorted block handled by the tensor-core path
-constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
-constexpr float kRescaleLog2 = 8.0f;   // rescale O only when the running max grows by more than this
-
-// MODE_DENSE: exact (non-causal) softmax attention of every query tile against every key chunk of its
-// sequence, with the CAUSAL mode's work layout (a "leaf" is the whole sequence) and no mask.
-enum { MODE_LEVEL = 0, MODE_CAUSAL = 1, MODE_DENSE = 2, MODE_LEVEL_RN = 3 };
-__host__ __device__ constexpr bool is_level(int mode) { return mode == MODE_LEVEL || mode == MODE_LEVEL_RN; }
-
-struct TcArgs {
-    int mode;
-    const uint16_t *Q, *K, *V;   // bf16 [bh * n][d]
-    int64_t n, bh;
-    // LEVEL
-    Level lv;
-    const int32_t *perm, *inv, *S;
-    int m;
-    int64_t nodes_total;
-    int nb, ns;            // block chunks, sample chunks
-    const int32_t *Srn;    // LEVEL_RN: row-norm draws [bh][nodes_total][m] (local key row, -1: none)
-    const float *lwrn;     // LEVEL_RN: their natural-log weights log(1 / (m p_j))
-    int nr;                // LEVEL_RN: row-norm chunks (0 otherwise)
-    int tiles_per_block, pairs_per_block;
-    float lw2;             // log2(N / m)
-    // CAUSAL
-    int64_t leaf, nleaves;
-    int levels, tiles_per_leaf, pairs_per_leaf;
-    const float *Opart_r, *Lpart_r;
-    // outputs
-    void *O;
-    int out_dtype;
-    float *lse, *Opart_w, *Lpart_w;
-    int *status;
-    int64_t stall_ns;      // test hook: > 0 makes the first softmax wait give up after this long (see bNever)
-    int64_t items;
-    uint32_t per_outer;    // LEVEL: items per problem; CAUSAL: items per query-tile pair index
-};
-
-struct Item {
-    bool v0, v1;          // tile validity
-    int nc0, nc1;         // key chunks of each tile (0 when invalid)
-    int nc_max, npairs;
-    // LEVEL
-    int64_t prob, blk, bhi, node;
-    int pair;
-    // CAUSAL
-    int64_t leaf_start;   // global row of the leaf's first row (bhi * n + leaf offset)
-    int gt0, gt1;         // query tile index within the leaf
-};
-
-// Item index -> item. Item counts, problem counts and their factors are below 2^31 (checked on the host), so the
-// divisions are 32-bit.
-template <int MODE>
-__device__ __forceinline__ Item decode(const TcArgs &a, int64_t it64) {
-    Item x{};
-    const uint32_t it = static_cast<uint32_t>(it64);
-    if (is_level(MODE)) {
-        const uint32_t prob = it / a.per_outer;
-        const uint32_t rem = it - prob * a.per_outer;
-        const uint32_t ppb = static_cast<uint32_t>(a.pairs_per_block);
-        const uint32_t blk = rem / ppb;
-        x.prob = prob;
-        x.blk = blk;
-        x.pair = static_cast<int>(rem - blk * ppb);
-        const uint32_t nodes = static_cast<uint32_t>(a.lv.nodes);
-        const uint32_t bhi = prob / nodes;
-        x.bhi = bhi;
-        x.node = prob - bhi * nodes;
-        x.v0 = x.pair * 2 < a.tiles_per_block;
-        x.v1 = x.pair * 2 + 1 < a.tiles_per_block;
-        x.nc0 = x.v0 ? a.nb + a.ns + a.nr : 0;
-        x.nc1 = x.v1 ? a.nb + a.ns + a.nr : 0;
-    } else {
-        const uint32_t po = it / a.per_outer;
-        const int pair = a.pairs_per_leaf - 1 - static_cast<int>(po);   // heaviest first
-        const uint32_t rem = it - po * a.per_outer;
-        const uint32_t nl = static_cast<uint32_t>(a.nleaves);
-        const uint32_t bhi = rem / nl;
-        x.bhi = bhi;
-        x.leaf_start = static_cast<int64_t>(bhi) * a.n + static_cast<int64_t>(rem - bhi * nl) * a.leaf;
-        x.pair = pair;
-        x.gt0 = pair * 2;
-        x.gt1 = pair * 2 + 1;
-        x.v0 = x.gt0 < a.tiles_per_leaf;
-        x.v1 = x.gt1 < a.tiles_per_leaf;
-        x.nc0 = x.v0 ? (MODE == MODE_DENSE ? a.tiles_per_leaf : x.gt0 + 1) : 0;
-        x.nc1 = x.v1 ? (MODE == MODE_DENSE ? a.tiles_per_leaf : x.gt1 + 1) : 0;
-    }
-    x.nc_max = max(x.nc0, x.nc1);
-    x.npairs = x.nc0 + x.nc1;
-    return x;
-}
-
-// Position of pair (t, c) in the item's pair order (c-major, t-minor, skipping finished tiles).
-__device__ __forceinline__ int pair_index(const Item &x, int t, int c) {
-    const int mn = min(x.nc0, x.nc1);
-    if (mn == 0) return c;
-    if (c < mn) return 2 * c + t;
-    return 2 * mn + (c - mn);
-}
-
-// Inverse of pair_index.
-__device__ __forceinline__ void pair_tc(const Item &x, int k, int &t, int &c) {
-    const int mn = min(x.nc0, x.nc1);
-    if (mn == 0) { t = x.v0 ? 0 : 1; c = k; return; }
-    if (k < 2 * mn) { t = k & 1; c = k >> 1; return; }
-    t = x.nc0 > x.nc1 ? 0 : 1;
-    c = mn + (k - 2 * mn);
-}
 
 template <int D>
 struct Cfg {
@@ -237,79 +124,6 @@ struct Cfg {
     static_assert(kOCol + 2 * D <= 512, "TMEM budget");
 };
 
-__device__ __forceinline__ void flag_status(int *status) {
-    if (status) atomicOr(status, kStatusTimeout);
-}
-
-// One SEG-byte segment, at byte offset `off`, of each of the warp's 32 output rows: lane l holds the segment of
-// its own row (16-byte pieces pc[0..SEG/16)) and `drow` points at the start of that row. The segments pass
-// through the warp's shared-memory stage (32 x SEG bytes, pieces XOR-swizzled so that neither the row-wise
-// writes nor the column-wise reads conflict on banks), so that SEG/16 consecutive lanes store one row's SEG
-// contiguous bytes: an instruction touches 32 / (SEG/16) rows instead of 32.
-template <int SEG>
-__device__ __forceinline__ void warp_store_segment(unsigned char *stage, unsigned char *drow, int off,
-                                                   const uint4 (&pc)[SEG / 16], int lane) {
-    constexpr int P = SEG / 16, SH = SEG == 64 ? 1 : 0;
-    __syncwarp();   // the previous segment's reads of the stage are done
-#pragma unroll
-    for (int j = 0; j < P; ++j)
-        *reinterpret_cast<uint4 *>(stage + lane * SEG + ((j ^ ((lane >> SH) & (P - 1))) << 4)) = pc[j];
-    __syncwarp();
-    const int sub = lane / P, piece = lane % P;
-#pragma unroll
-    for (int i = 0; i < P; ++i) {
-        const int row = i * (32 / P) + sub;
-        const uint4 v = *reinterpret_cast<const uint4 *>(stage + row * SEG + ((piece ^ ((row >> SH) & (P - 1))) << 4));
-        unsigned char *rb = reinterpret_cast<unsigned char *>(
-            __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(drow), row));
-        *reinterpret_cast<uint4 *>(rb + off + piece * 16) = v;
-    }
-}
-
-// Write the warp's 32 rows of D output values (bf16 or fp32; lane l owns row l at `drow`). vals(j, v) yields
-// the row's columns [32 j, 32 j + 32) as floats.
-template <int D, int SEG, typename F>
-__device__ __forceinline__ void warp_write_rows(unsigned char *stage, unsigned char *drow, bool bf16, int lane,
-                                                F &&vals) {
-    constexpr int PS = SEG / 16;
-    uint4 seg[PS];
-    if (bf16) {
-#pragma unroll
-        for (int j = 0; j < D / 32; ++j) {
-            float v[32];
-            vals(j, v);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int pi = j * 4 + q;
-                seg[pi % PS] = make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                                          pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
-                if (pi % PS == PS - 1) warp_store_segment<SEG>(stage, drow, (pi / PS) * SEG, seg, lane);
-            }
-        }
-    } else {
-#pragma unroll
-        for (int j = 0; j < D / 32; ++j) {
-            float v[32];
-            vals(j, v);
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const int pi = j * 8 + q;
-                seg[pi % PS] = make_uint4(__float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
-                                          __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3]));
-                if (pi % PS == PS - 1) warp_store_segment<SEG>(stage, drow, (pi / PS) * SEG, seg, lane);
-            }
-        }
-    }
-}
-
-// byte offset of 16-byte piece j of row `row` inside a 128-row, 128-byte-swizzled tile (slab s = 64 columns)
-__device__ __forceinline__ uint32_t swz(int slab, int row, int j) {
-    return static_cast<uint32_t>(slab * (128 * 128) + row * 128 + ((j ^ (row & 7)) << 4));
-}
-
-// MODE (MODE_LEVEL, MODE_LEVEL_RN, MODE_CAUSAL or MODE_DENSE) is a compile-time parameter: each instance holds
-// only its own mode's loads,
-// masks and epilogue, which keeps the instruction footprint of the concurrently running roles small (measured:
 // about 4% faster than one instance for both modes).
 template <int D, int MODE, bool HOOK>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
@@ -377,14 +191,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
         stride = gridDim.x;
     }
 
-    constexpr int PPR = D / 8;             // 16-byte pieces per row
-    constexpr int RPI = 32 / PPR;          // rows per warp instruction
 
     // Q tiles: tile t of an item into Q buffer qc mod QB of that tile, after the buffer's previous user (the
     // tile's score products and, with the epilogue staged there, its epilogue) is done with it
     int qc0 = 0, qc1 = 0;
     auto load_q_tile = [&](const Item &x, int t) -> bool {
-        const int rsub = lane / PPR, piece = lane % PPR, slab = piece >> 3, jp = piece & 7;
         int32_t *qperm = reinterpret_cast<int32_t *>(sm + C::kQPerm);
         int &qc = t == 0 ? qc0 : qc1;
         const int qb = qc % C::QB;
@@ -405,12 +216,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
         } else {
             qbase = x.leaf_start + static_cast<int64_t>(t == 0 ? x.gt0 : x.gt1) * 128;
         }
-#pragma unroll 8
-        for (int r0 = 0; r0 < 128; r0 += RPI) {
-            const int row = r0 + rsub;
-            const int64_t grow = qbase + (through_perm ? qperm[row] : row);
-            cp_async16(base + swz(slab, row, jp), a.Q + grow * D + piece * 8);
-        }
+        if (through_perm) gather_rows<D, true>(base, a.Q, qbase, qperm, lane);
+        else gather_rows<D, false>(base, a.Q, qbase, qperm, lane);
         cp_async_arrive(bar(C::bQFull + t * C::QB + qb));
         ++qc;
         return true;
@@ -428,7 +235,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
         if (!ok) flag_status(a.status);
     } else if (warp == 0) {
         // ------------------------------------------------------------------ K/V loader
-        const int rsub = lane / PPR, piece = lane % PPR, slab = piece >> 3, jp = piece & 7;
         const unsigned lt_mask = (1u << lane) - 1u;
         int32_t *slist = reinterpret_cast<int32_t *>(sm + C::kList);
         int32_t *cache_s = reinterpret_cast<int32_t *>(sm + C::kCacheS);
@@ -551,11 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(C::bRowsFull + slot));
                 const uint32_t kb = sbase + C::kK + slot * C::kTileBytes;
-#pragma unroll 8
-                for (int r0 = 0; r0 < kKC; r0 += RPI) {
-                    const int row = r0 + rsub;
-                    cp_async16(kb + swz(slab, row, jp), a.K + static_cast<int64_t>(rows[row]) * D + piece * 8);
-                }
+                gather_rows<D, true>(kb, a.K, 0, rows, lane);
                 cp_async_arrive(bar(C::bKVFull + slot));
             }
         }
@@ -564,7 +366,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
     } else if (warp == 3) {
         // ------------------------------------------------------------------ V loader
         // follows the K loader's chunk sequence: waits for each stage's row list, copies the V rows
-        const int rsub = lane / PPR, piece = lane % PPR, slab = piece >> 3, jp = piece & 7;
         const int32_t *stage_rows = reinterpret_cast<const int32_t *>(sm + C::kRows);
         uint32_t g = 0;
         bool ok = true;
@@ -580,11 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                 }
                 const int32_t *rows = stage_rows + slot * 128;
                 const uint32_t vb = sbase + C::kV + slot * C::kTileBytes;
-#pragma unroll 8
-                for (int r0 = 0; r0 < kKC; r0 += RPI) {
-                    const int row = r0 + rsub;
-                    cp_async16(vb + swz(slab, row, jp), a.V + static_cast<int64_t>(rows[row]) * D + piece * 8);
-                }
+                gather_rows<D, true>(vb, a.V, 0, rows, lane);
                 cp_async_arrive(bar(C::bKVFull + slot));
             }
         }
@@ -1195,6 +992,15 @@ int launch_tc(const void *Q, const void *K, const void *V, TcArgs args, cudaStre
 }
 
 int dispatch(int d, const void *Q, const void *K, const void *V, const TcArgs &args, cudaStream_t st) {
+    {
+        // the single-tile kernel of ha_attn_pp.cu for the modes and head dims it covers
+        TcArgs pa = args;
+        pa.Q = static_cast<const uint16_t *>(Q);
+        pa.K = static_cast<const uint16_t *>(K);
+        pa.V = static_cast<const uint16_t *>(V);
+        const int k = launch_attn_pp(d, pa, num_sms(), st);
+        if (k != -2) return k;
+    }
     const bool level = args.mode == MODE_LEVEL;
     const bool dense = args.mode == MODE_DENSE;
     if (args.mode == MODE_LEVEL_RN) {

@@ -97,6 +97,22 @@ def algorithmic(w: wl.Workload, cls: str, sampling: str = "uniform"):
     raise KeyError(cls)
 
 
+def step_work(w: wl.Workload):
+    """The method's algorithmic work of one whole forward pass (all heads): (bytes, flops). Non-causal per head:
+    reads of Q and K for the hash, of Q, K and V for the attention, the write of O, and 32 bytes per row of ranks and
+    permutations; 4 n d (b + m) flops for the two contractions. Causal per head: the exact leaves (2 n d c flops) plus
+    L levels of the non-causal problem on half the rows, each with its part written and read back once."""
+    e = 2 if w.dtype == "bf16" else 4
+    n, d, bh = w.n, w.d, w.bh
+    if not w.causal:
+        return bh * (6.0 * n * d * e + 32.0 * n), bh * 4.0 * n * d * (min(w.block, n) + w.m)
+    L = nlev_of(w)
+    c = min(w.base, n)
+    flops = bh * 2.0 * n * d * (c + L * (w.block + w.m))
+    byts = bh * ((6.0 * n * d + 1.5 * L * n * d) * e + 32.0 * n * (L + 1))
+    return byts, flops
+
+
 class ClockSampler:
     """Samples SM clock, power and clock-event reasons of one GPU with NVML while running."""
 
@@ -185,6 +201,23 @@ def cpu_oracle_rate(w: wl.Workload, heads, sampling="uniform"):
                        causal=w.causal, base=w.base, seed=w.algo_seed, bh=h, sampling=sampling)
     dt = time.perf_counter() - t0
     return len(heads) * w.n / dt / 1e6, dt, oracle.num_threads()
+
+
+def parity_spot(w: wl.Workload, out_head0, sampling="uniform", nrows: int = 64, seed: int = 11):
+    """The oracle on seeded rows of head 0, against the timed run's output of those rows (part of the CPU-baseline
+    leg, after the timed region). The output has the input's type, so a bf16 output adds its own rounding (2^-9
+    relative) to the parity tolerance (2e-3 for bf16 inputs, 1e-4 for fp32)."""
+    import oracle
+    oracle.build()
+    Qh, Kh, Vh = wl.workload_inputs(w, heads=[0])
+    rows = np.sort(np.random.default_rng(seed).choice(w.n, size=min(nrows, w.n), replace=False))
+    ref = oracle.forward(wl.as_f32(Qh[0]), wl.as_f32(Kh[0]), wl.as_f32(Vh[0]), block=w.block, m=w.m, r=w.r,
+                         causal=w.causal, base=w.base, seed=w.algo_seed, bh=0, rows=rows, sampling=sampling)["O"]
+    got = out_head0[rows]
+    err = float(np.linalg.norm(got - ref) / np.linalg.norm(ref))
+    tol = 2e-3 + 2.0 ** -9 if w.dtype == "bf16" else 1e-4
+    return {"rows": int(len(rows)), "head": 0, "rel_l2": err, "tol": tol, "pass": bool(err < tol),
+            "vs": "oracle on the same seeded inputs and draws (timed run's output)"}
 
 
 def run_reference(args, w: wl.Workload):
@@ -323,6 +356,7 @@ def run_ours(args, w: wl.Workload):
     ha.profile(False)
     prof = ha.profile_read()
     assert ha.status() == 0, ha.last_error()
+    out_head0 = O[0].float().cpu().numpy().astype(np.float64) if rank == 0 else None   # for the spot check
     ms = ev0.elapsed_time(ev1) / args.steps
     ms_max = max_over_ranks(ms, dev)
     units = world * w.bh * w.n
@@ -445,17 +479,29 @@ def run_ours(args, w: wl.Workload):
         if os.path.exists(src) and hashlib.sha256(open(src, "rb").read()).hexdigest() == tr["sha256"]:
             traffic = tr["bytes"]
 
+    sbytes, sflops = step_work(w)
+    cpk = peaks["bf16_tflops"] if family == "tc" else FP32_SIMT_PEAK_TFLOPS
+    t_hbm = sbytes / (peaks["hbm_gbs"] * 1e9) * 1e3
+    t_cmp = sflops / (cpk * 1e12) * 1e3
+    roof_step = {"t_roof_ms": max(t_hbm, t_cmp), "frac": max(t_hbm, t_cmp) / ms_max,
+                 "bound": ("hbm" if t_hbm >= t_cmp else ("tensor" if family == "tc" else "alu")),
+                 "bytes": sbytes, "flops": sflops, "t_hbm_ms": t_hbm, "t_compute_ms": t_cmp,
+                 "peak_source": peak_src + (" burst" if family == "tc" else ""),
+                 "note": "whole forward step (all kernels) against the method's algorithmic bytes and flops"}
+
     err = None
     if rank == 0:
         f64 = lambda t: t.float().numpy().astype(np.float64)
         err = approx_error(f64(hQ[0]), f64(hK[0]), f64(hV[0]), f64(hO[0]), w.causal)
 
     cpu = None
+    spot = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         heads = list(range(min(args.cpu_heads, w.bh)))
         rate, secs, cores = cpu_oracle_rate(w, heads, args.sampling)
         cpu = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": f"{len(heads)} of {w.bh} heads, all {w.n} query rows ({secs:.1f} s)"}
+        spot = parity_spot(w, out_head0, args.sampling)
 
     if rank == 0:
         line = {
@@ -467,12 +513,14 @@ def run_ours(args, w: wl.Workload):
                          "frac": achieved / peak, "traffic": traffic, "kernel": dom,
                          "kernel_ms_per_launch": avg_ms, "peak_source": peak_src + (" burst" if bound == "tensor" else ""),
                          "kernel_family": "tcgen05" if family == "tc" else "simt"},
+            "roofline_step": roof_step,
             "kernel_ms_per_step": {k: v[0] / args.steps for k, v in prof.items()},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": 3 * Q.numel() * esz,
                     "d2h_bytes_per_step": O.numel() * esz},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk.summary(),
             "cpu_baseline": cpu,
+            "parity_spot": spot,
             "approx_error": err,
             "vs_exact": vs_exact,
         }

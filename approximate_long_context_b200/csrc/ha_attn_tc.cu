@@ -74,11 +74,6 @@ struct Cfg {
     // product from queueing right behind the P.V that reads its buffer (a tensor-pipe stall; d = 128 is bound
     // by the pipe), one gives the second tile its next score tile sooner (d = 64 is bound by the softmax)
     static constexpr int kGroup = D == 64 ? 1 : 2;
-    // Two MMA issuers (score products on warp 1, P.V products on warp 2, the K loader also loading the Q
-    // tiles) instead of one issuer for both and a Q loader. Measured slower on this part for both head dims
-    // (a score product then waits for the completion of the P.V that last read its buffer, instead of queueing
-    // behind it), so it is off; the code is kept for other shapes and parts.
-    static constexpr bool kSplit = false;
     static constexpr int SEG = D == 64 ? 128 : 64;     // bytes per row segment of the staged output stores
     // d = 64: the epilogue stages its output rows in the item's own Q buffer (dead once the tile's last score
     // product has completed; the Q loader refills it only after the epilogue); d = 128 has a stage of its own
@@ -223,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
         return true;
     };
 
-    if (warp == 2 && !C::kSplit) {
+    if (warp == 2) {
         // ------------------------------------------------------------------ Q loader
         bool ok = true;
         for (int64_t it = first; it < last && ok; it += stride) {
@@ -249,11 +244,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
         bool ok = true;
         for (int64_t it = first; it < last && ok; it += stride) {
             const Item x = decode<MODE>(a, it);
-            if (C::kSplit) {   // this warp also loads the Q tiles (their buffers wait on items two back)
-                if (x.v0) ok = load_q_tile(x, 0);
-                if (ok && x.v1) ok = load_q_tile(x, 1);
-                if (!ok) break;
-            }
             // key rows of block blk and the compacted sample list of this item: the sampled columns whose key
             // lies outside block blk, in sample order (from the per-problem cache of samples and their blocks)
             int cnt = 0, cnt_rn = 0;
@@ -387,7 +377,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
         }
         cp_wait<0>();
         if (!ok) flag_status(a.status);
-    } else if (warp == 1 && !C::kSplit) {
+    } else if (warp == 1) {
         // ------------------------------------------------------------------ MMA issuer (score and P.V products)
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16(128, kKC, false, false);
@@ -545,119 +535,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
             mma_commit(bar(C::bDrain));   // every MMA issued so far completes before TMEM is released
             volatile int no_abort = 0;
             mbar_wait(bar(C::bDrain), 0, &no_abort, 200000000ull);
-        }
-        __syncwarp();
-    } else if (warp == 1 && C::kSplit) {
-        // ------------------------------------------------------------------ score MMA issuer
-        // S of pair j (pair count of this CTA over all items) goes to ring buffer j mod R once P.V of pair j - R,
-        // the buffer's previous reader, has completed; runs ahead across items as far as the ring, the Q buffers
-        // and the K/V stages allow.
-        if (lane == 0) {
-            constexpr uint32_t idesc_qk = idesc_bf16(128, kKC, false, false);
-            // descriptors are built once; an MMA only adds a byte offset >> 4 to the start-address field
-            const uint64_t dq0 = smem_desc(sbase + C::kQ, 16, 1024);
-            const uint64_t dk0 = smem_desc(sbase + C::kK, 16, 1024);
-            uint32_t j = 0, g = 0, kv_ready = 0;
-            int sq0 = 0, sq1 = 0;   // Q tiles taken per tile
-            bool ok = true;
-            for (int64_t it = first; it < last && ok; it += stride) {
-                const Item x = decode<MODE>(a, it);
-                int qb0 = -1, qb1 = -1;
-                for (int k = 0; k < x.npairs; ++k, ++j) {
-                    int t, c;
-                    pair_tc(x, k, t, c);
-                    int &qb = t == 0 ? qb0 : qb1;
-                    if (qb < 0) {
-                        int &qc = t == 0 ? sq0 : sq1;
-                        if (!mbar_wait(bar(C::bQFull + t * C::QB + qc % C::QB), (qc / C::QB) & 1, abort_flag)) {
-                            ok = false;
-                            break;
-                        }
-                        qb = qc % C::QB;
-                        ++qc;
-                    }
-                    const uint32_t gc = g + static_cast<uint32_t>(c);
-                    const int slot = static_cast<int>(gc % C::NST);
-                    if (gc >= kv_ready) {   // chunks arrive in order: wait once per chunk
-                        if (!mbar_wait(bar(C::bKVFull + slot), (gc / C::NST) & 1, abort_flag)) { ok = false; break; }
-                        kv_ready = gc + 1;
-                    }
-                    const int buf = static_cast<int>(j % C::R);
-                    if (j >= static_cast<uint32_t>(C::R) &&
-                        !mbar_wait(bar(C::bPVDone + buf), (j / C::R - 1) & 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint64_t dq = dq0 + static_cast<uint64_t>(((t * C::QB + qb) * C::kTileBytes) >> 4);
-                    const uint64_t dk = dk0 + static_cast<uint64_t>((slot * C::kTileBytes) >> 4);
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint64_t off = static_cast<uint64_t>(((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4);
-                        mma_ss(tmem + buf * 128, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
-                    }
-                    mma_commit(bar(C::bSFull + buf));
-                    // last score tile of this query tile in this item: its Q buffer may be refilled
-                    if (c == (t == 0 ? x.nc0 : x.nc1) - 1) mma_commit(bar(C::bQEmpty + t * C::QB + qb));
-                }
-                g += static_cast<uint32_t>(x.nc_max);
-            }
-            if (!ok) flag_status(a.status);
-            mma_commit(bar(C::bDrain));   // this thread's MMAs complete before TMEM is released
-            volatile int no_abort = 0;
-            mbar_wait(bar(C::bDrain), 0, &no_abort, 200000000ull);
-        }
-        __syncwarp();
-    } else if (warp == 2 && C::kSplit) {
-        // ------------------------------------------------------------------ P.V MMA issuer
-        // O_t += P(j) V(chunk) once the softmax has written P of pair j; then signals the tile's P.V count
-        // (softmax: rescale and epilogue), the ring buffer (score issuer) and, after the chunk's last user, the
-        // K/V stage.
-        if (lane == 0) {
-            constexpr uint32_t idesc_pv = idesc_bf16(128, D, false, true);
-            const uint64_t dv0 = smem_desc(sbase + C::kV, 128 * 128, 1024);
-            uint32_t j = 0, g = 0;
-            uint32_t pvn0 = 0, pvn1 = 0;   // P.V products issued per tile
-            int oc0 = 0, oc1 = 0;
-            bool ok = true;
-            for (int64_t it = first; it < last && ok; it += stride) {
-                const Item x = decode<MODE>(a, it);
-                for (int k = 0; k < x.npairs; ++k, ++j) {
-                    int t, c;
-                    pair_tc(x, k, t, c);
-                    const int buf = static_cast<int>(j % C::R);
-                    if (!mbar_wait(bar(C::bPFull + buf), (j / C::R) & 1, abort_flag)) { ok = false; break; }
-                    const int oc = t == 0 ? oc0 : oc1;
-                    if (c == 0 && oc > 0 && !mbar_wait(bar(C::bOFree + t), (oc - 1) & 1, abort_flag)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t gc = g + static_cast<uint32_t>(c);
-                    const int slot = static_cast<int>(gc % C::NST);
-                    // V of chunk c arrived with K (one barrier per stage), which S of this pair waited for
-                    const uint64_t dv = dv0 + static_cast<uint64_t>((slot * C::kTileBytes) >> 4);
-                    const uint32_t od = tmem + C::kOCol + t * D;
-                    if (MODE != MODE_LEVEL_RN || c < a.nb || c >= a.nb + a.ns) {
-#pragma unroll
-                        for (int kk = 0; kk < kKC / 16; ++kk)
-                            mma_ts(od, tmem + buf * 128 + kk * 8, dv + static_cast<uint64_t>((kk * 2048) >> 4),
-                                   idesc_pv, (c > 0 || kk > 0) ? 1u : 0u);
-                    }
-                    // the tile's barrier first, then the ring buffer's: a waiter that has seen the buffer free may
-                    // rely on the tile's barrier having arrived
-                    uint32_t &pvn = t == 0 ? pvn0 : pvn1;
-                    mma_commit(bar(C::bPVDoneT + 2 * t + (pvn & 1)));
-                    ++pvn;
-                    mma_commit(bar(C::bPVDone + buf));
-                    // the chunk's stage is free once every tile that uses it has issued its P.V
-                    if (t == 1 || c >= x.nc1) mma_commit(bar(C::bKVEmpty + slot));
-                }
-                if (x.v0) ++oc0;
-                if (x.v1) ++oc1;
-                g += static_cast<uint32_t>(x.nc_max);
-            }
-            if (!ok) flag_status(a.status);
-            mma_commit(bar(C::bDrain + 1));
-            volatile int no_abort = 0;
-            mbar_wait(bar(C::bDrain + 1), 0, &no_abort, 200000000ull);
         }
         __syncwarp();
     } else if (warp >= 4) {

@@ -1,11 +1,10 @@
 // ha_sm100.cuh -- thin inline-PTX wrappers for the sm_100a features the tensor-core kernels use:
-// mbarriers (with bounded waits), TMA tensor loads (tile and tile::gather4, never multicast), and the
+// mbarriers (with bounded waits), 16-byte cp.async copies, and the
 // tcgen05 family (TMEM allocation, MMA, commit, TMEM loads and stores, fences).
 // Written from the PTX ISA; descriptor bit layouts follow the sm_100 UMMA shared-memory and instruction
 // descriptor definitions.
 #pragma once
 
-#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -99,32 +98,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
                                           uint64_t limit_ns = 2000000000ull) {
     if (__builtin_expect(mbar_try_wait(bar, parity), 1)) return true;
     return mbar_wait_slow(bar, parity, abort, limit_ns);
-}
-
-// --------------------------------------------------------------------------------------------- TMA
-
-// Four rows (row0..row3 of a 2-D tensor map whose box is {box_cols, 1}) starting at column `col` into
-// consecutive box-sized pieces of shared memory at `dst`; completion is counted on `bar` in bytes.
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap *map, int col, int row0, int row1,
-                                            int row2, int row3, uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(col), "r"(row0), "r"(row1), "r"(row2), "r"(row3), "r"(bar)
-        : "memory");
-}
-
-// One box of a 2-D tensor map at (col, row) into shared memory at `dst`.
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int col, int row, uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(col), "r"(row), "r"(bar)
-        : "memory");
-}
-
-__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
 // ------------------------------------------------------------------------------- cp.async (LDGSTS)

@@ -53,6 +53,7 @@ constexpr int kRegsOther = 104;     // loader/issuer and epilogue warpgroups
 static_assert(128 * (2 * kRegsSoftmax + 2 * kRegsOther) == kSTThreads * 128,
               "the warpgroups' budgets add up to the launch's registers");
 constexpr int kCK = 128;            // keys per chunk
+constexpr int kMaxItemChunks = kMaxBlock / kCK + kMaxSampleList / kCK;   // block chunks + sample chunks of an item
 
 struct STCfg {
     static constexpr int D = 64;
@@ -71,13 +72,15 @@ struct STCfg {
     static constexpr int kCacheB = kCacheS + kMaxSampleList * 4;          // their sorted key block
     static constexpr int kKPerm = kCacheB + kMaxSampleList * 4;           // key rows of the current block
     static constexpr int kQPerm = kKPerm + kMaxBlock * 4;                 // query rows of one tile
-    static constexpr int kRows = kQPerm + 128 * 4;                        // global rows of each stage
-    static constexpr int kStats = kRows + NST * kCK * 4;                  // [item parity][half][row]: max, sum
+    static constexpr int kIList = kQPerm + 128 * 4;                       // [item parity]: global key rows per chunk
+    static constexpr int kIWord = kIList + 2 * kMaxItemChunks * kCK * 4;  // [item parity]: valid columns per chunk
+    static constexpr int kStats = kIWord + 2 * kMaxItemChunks * 4;        // [item parity][half][row]: max, sum
     static constexpr int kXch = kStats + 2 * 2 * 128 * 8;                 // [chunk parity][half][row]: partial maxima
     static constexpr int kWord = kXch + 2 * 2 * 128 * 4;
     static constexpr int kBars = (kWord + NST * 4 + 15) / 16 * 16;
     static constexpr int bQFull = 0, bQEmpty = bQFull + QB, bKVFull = bQEmpty + QB, bKVEmpty = bKVFull + NST,
-                         bWordFull = bKVEmpty + NST, bRowsFull = bWordFull + NST, bSFull = bRowsFull + NST,
+                         bWordFull = bKVEmpty + NST, bListFull = bWordFull + NST, bListEmpty = bListFull + 2,
+                         bSFull = bListEmpty + 2,
                          bPFull = bSFull + 2, bPVDone = bPFull + 2, bOReady = bPVDone + 2, bOFree = bOReady + 2,
                          bStatsReady = bOFree + 2, bStatsFree = bStatsReady + 2, bDrain = bStatsFree + 2,
                          kNumBars = bDrain + 1;
@@ -136,6 +139,25 @@ __device__ __forceinline__ Tile decode_tile(const TcArgs &a, int64_t it64) {
     return x;
 }
 
+// P = 2^(s log2(e) + off) over this half's 64 columns, rounded to bf16 pairs; returns the row sum of P (of the fp32
+// values). The scale-and-offset and the sums run as packed f32x2 instructions (half the issue slots of scalar ones);
+// the exponentials on the MUFU unit. Masked columns (s = -inf) give 2^-inf = 0.
+__device__ __forceinline__ float exp_half(const uint32_t (&v)[64], float off, uint32_t (&pk)[32]) {
+    const uint64_t sc = f2_pack(kLog2e, kLog2e), of = f2_pack(off, off);
+    uint64_t la = f2_pack(0.0f, 0.0f), lb = la;
+#pragma unroll
+    for (int e = 0; e < 64; e += 2) {
+        const float2 x = f2_unpack(f2_fma(f2_pack(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), sc, of));
+        const float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
+        const uint64_t p = f2_pack(p0, p1);
+        if (e & 2) lb = f2_add(lb, p);
+        else la = f2_add(la, p);
+        pk[e / 2] = pack_bf16x2(p0, p1);
+    }
+    const float2 l2 = f2_unpack(f2_add(la, lb));
+    return l2.x + l2.y;
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) {
     using C = STCfg;
@@ -161,7 +183,10 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
             mbar_init(bar(C::bKVFull + s), 64);    // the K and V loader warps' lanes (copy completion)
             mbar_init(bar(C::bKVEmpty + s), 1);    // commit after the chunk's P.V product
             mbar_init(bar(C::bWordFull + s), 1);
-            mbar_init(bar(C::bRowsFull + s), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar(C::bListFull + i), 1);   // the list builder: an item's key rows and column counts written
+            mbar_init(bar(C::bListEmpty + i), 2);  // the K and V loaders: done with the item's list
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar(C::bSFull + b), 1);      // commit after a score product into S_b
@@ -206,59 +231,35 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
     if (warp < 4) {
         setmaxnreg_dec<kRegsOther>();
         if (warp == 2) {
-            // -------------------------------------------------------------- Q loader
-            // item i's tile into Q buffer i mod QB, once the buffer's previous tile has issued its last score product
-            // (the commit after it arrives on the buffer's "empty" barrier)
-            int32_t *qperm = reinterpret_cast<int32_t *>(sm + C::kQPerm);
-            int qc = 0;
-            bool ok = true;
-            for (int64_t it = first; it < last && ok; it += stride, ++qc) {
-                const Tile x = decode_tile<MODE>(a, it);
-                const int qb = qc % C::QB, use = qc / C::QB;
-                if (use > 0 && !mbar_wait_inl(bar(C::bQEmpty + qb), (use - 1) & 1, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                const uint32_t base = sbase + C::kQ + qb * C::kQBytes;
-                if (is_level(MODE)) {
-                    const int32_t *pq = a.perm + (static_cast<int64_t>(x.prob) * 2) * a.lv.seg_len +
-                                        static_cast<int64_t>(x.blk) * a.lv.bp + x.tile * 128;
-                    __syncwarp();
-                    reinterpret_cast<int4 *>(qperm)[lane] = reinterpret_cast<const int4 *>(pq)[lane];
-                    __syncwarp();
-                    gather_rows<D, true>(base, a.Q,
-                                         static_cast<int64_t>(x.bhi) * a.n + static_cast<int64_t>(x.node) * a.lv.node_len +
-                                             a.lv.q_off,
-                                         qperm, lane);
-                } else {
-                    gather_rows<D, false>(base, a.Q, x.leaf_start + static_cast<int64_t>(x.gt) * 128, qperm, lane);
-                }
-                cp_async_arrive(bar(C::bQFull + qb));
-            }
-            cp_wait<0>();
-            if (!ok) flag_status(a.status);
-        } else if (warp == 0) {
-            // -------------------------------------------------------------- K loader
-            // chunk g of the CTA (over all items) goes to stage g mod NST once the stage's previous chunk has
-            // completed its products; the stage's row list is published for the V loader
+            // -------------------------------------------------------------- list builder and Q loader
+            // Per item i: the global key rows of all its chunks and their valid column counts into list slot
+            // i mod 2 (once the loaders are done with item i - 2), then the query tile into Q buffer i mod QB (once
+            // the buffer's previous tile has issued its last score product). The lists run an item ahead of the
+            // loaders, so the loaders only copy rows.
             const unsigned lt_mask = (1u << lane) - 1u;
             int32_t *slist = reinterpret_cast<int32_t *>(sm + C::kList);
             int32_t *cache_s = reinterpret_cast<int32_t *>(sm + C::kCacheS);
             int32_t *cache_b = reinterpret_cast<int32_t *>(sm + C::kCacheB);
             int32_t *kperm = reinterpret_cast<int32_t *>(sm + C::kKPerm);
-            int32_t *stage_rows = reinterpret_cast<int32_t *>(sm + C::kRows);
+            int32_t *qperm = reinterpret_cast<int32_t *>(sm + C::kQPerm);
             int64_t cached_prob = -1, cached_blk = -1;
             int cnt = 0;
-            uint32_t g = 0;
+            uint32_t ni = 0;
             bool ok = true;
-            for (int64_t it = first; it < last && ok; it += stride) {
+            for (int64_t it = first; it < last && ok; it += stride, ++ni) {
                 const Tile x = decode_tile<MODE>(a, it);
+                const int ls = static_cast<int>(ni & 1);
+                if (ni >= 2 && !mbar_wait_inl(bar(C::bListEmpty + ls), ((ni >> 1) - 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                int32_t *ilist = reinterpret_cast<int32_t *>(sm + C::kIList) + ls * (kMaxItemChunks * kCK);
+                int32_t *iword = reinterpret_cast<int32_t *>(sm + C::kIWord) + ls * kMaxItemChunks;
                 int64_t kbase = 0;
                 if (is_level(MODE)) {
                     kbase = static_cast<int64_t>(x.bhi) * a.n + static_cast<int64_t>(x.node) * a.lv.node_len;
                     const int64_t key_blk = static_cast<int64_t>(x.prob) * (a.lv.seg_len / a.lv.bp) + x.blk;
                     if (key_blk != cached_blk) {
-                        // the stages still in use read their row lists, not these arrays: refill them
                         const int32_t *pkg = a.perm + (static_cast<int64_t>(x.prob) * 2 + 1) * a.lv.seg_len +
                                              static_cast<int64_t>(x.blk) * a.lv.bp;
                         __syncwarp();
@@ -290,24 +291,13 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
                         __syncwarp();
                     }
                 }
-                for (int c = 0; c < x.nc; ++c, ++g) {
-                    const int slot = static_cast<int>(g % C::NST);
-                    const uint32_t round = g / C::NST;
-                    if (round > 0 && !mbar_wait_inl(bar(C::bKVEmpty + slot), (round - 1) & 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    // LEVEL: chunks [0, ns) are sample chunks, [ns, ns + nb) block chunks
-                    int valid_cols = kCK;
+                // LEVEL: chunks [0, ns) are sample chunks (their tails, past the block's count, point at the first
+                // key row and are masked), [ns, ns + nb) block chunks
+                for (int c = 0; c < x.nc; ++c) {
                     const bool sample = is_level(MODE) && c < a.ns;
                     const int u0 = c * kCK;
-                    if (sample) valid_cols = min(kCK, max(0, cnt - u0));
-                    if (lane == 0) {
-                        words[slot] = valid_cols;
-                        mbar_arrive(bar(C::bWordFull + slot));
-                    }
+                    if (lane == 0) iword[c] = sample ? min(kCK, max(0, cnt - u0)) : kCK;
                     const int64_t cbase = is_level(MODE) ? kbase : x.leaf_start + static_cast<int64_t>(c) * kCK;
-                    int32_t *rows = stage_rows + slot * kCK;
 #pragma unroll
                     for (int rr = 0; rr < kCK / 32; ++rr) {
                         const int row = rr * 32 + lane;
@@ -315,29 +305,68 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
                         if (!is_level(MODE)) loc = row;
                         else if (sample) loc = row + u0 < cnt ? slist[u0 + row] : 0;
                         else loc = kperm[(c - a.ns) * kCK + row];
-                        rows[row] = static_cast<int32_t>(cbase + loc);
+                        ilist[c * kCK + row] = static_cast<int32_t>(cbase + loc);
                     }
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar(C::bRowsFull + slot));
-                    gather_rows<D, true, kCK>(sbase + C::kK + slot * C::kCBytes, a.K, 0, rows, lane);
-                    cp_async_arrive(bar(C::bKVFull + slot));
                 }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(C::bListFull + ls));
+                // the query tile
+                const int qb = static_cast<int>(ni % C::QB), use = static_cast<int>(ni / C::QB);
+                if (use > 0 && !mbar_wait_inl(bar(C::bQEmpty + qb), (use - 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t base = sbase + C::kQ + qb * C::kQBytes;
+                if (is_level(MODE)) {
+                    const int32_t *pq = a.perm + (static_cast<int64_t>(x.prob) * 2) * a.lv.seg_len +
+                                        static_cast<int64_t>(x.blk) * a.lv.bp + x.tile * 128;
+                    __syncwarp();
+                    reinterpret_cast<int4 *>(qperm)[lane] = reinterpret_cast<const int4 *>(pq)[lane];
+                    __syncwarp();
+                    gather_rows<D, true>(base, a.Q,
+                                         static_cast<int64_t>(x.bhi) * a.n + static_cast<int64_t>(x.node) * a.lv.node_len +
+                                             a.lv.q_off,
+                                         qperm, lane);
+                } else {
+                    gather_rows<D, false>(base, a.Q, x.leaf_start + static_cast<int64_t>(x.gt) * 128, qperm, lane);
+                }
+                cp_async_arrive(bar(C::bQFull + qb));
             }
             cp_wait<0>();
             if (!ok) flag_status(a.status);
-        } else if (warp == 3) {
-            // -------------------------------------------------------------- V loader
-            const int32_t *stage_rows = reinterpret_cast<const int32_t *>(sm + C::kRows);
-            uint32_t g = 0;
+        } else if (warp == 0 || warp == 3) {
+            // -------------------------------------------------------------- K loader (warp 0), V loader (warp 3)
+            // chunk g of the CTA (over all items) goes to stage g mod NST once the stage's previous chunk has
+            // completed its products; rows from the item's list. The K loader also publishes the chunk's valid
+            // column count for the softmax.
+            const bool is_k = warp == 0;
+            const uint16_t *src = is_k ? a.K : a.V;
+            const uint32_t dst0 = sbase + (is_k ? C::kK : C::kV);
+            uint32_t g = 0, ni = 0;
             bool ok = true;
-            for (int64_t it = first; it < last && ok; it += stride) {
+            for (int64_t it = first; it < last && ok; it += stride, ++ni) {
                 const Tile x = decode_tile<MODE>(a, it);
+                const int ls = static_cast<int>(ni & 1);
+                if (!mbar_wait_inl(bar(C::bListFull + ls), (ni >> 1) & 1, abort_flag)) { ok = false; break; }
+                const int32_t *ilist = reinterpret_cast<const int32_t *>(sm + C::kIList) + ls * (kMaxItemChunks * kCK);
+                const int32_t *iword = reinterpret_cast<const int32_t *>(sm + C::kIWord) + ls * kMaxItemChunks;
                 for (int c = 0; c < x.nc; ++c, ++g) {
                     const int slot = static_cast<int>(g % C::NST);
-                    if (!mbar_wait_inl(bar(C::bRowsFull + slot), (g / C::NST) & 1, abort_flag)) { ok = false; break; }
-                    gather_rows<D, true, kCK>(sbase + C::kV + slot * C::kCBytes, a.V, 0, stage_rows + slot * kCK, lane);
+                    const uint32_t round = g / C::NST;
+                    if (round > 0 && !mbar_wait_inl(bar(C::bKVEmpty + slot), (round - 1) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    if (is_k && lane == 0) {
+                        words[slot] = iword[c];
+                        mbar_arrive(bar(C::bWordFull + slot));
+                    }
+                    gather_rows<D, true, kCK>(dst0 + slot * C::kCBytes, src, 0, ilist + c * kCK, lane);
                     cp_async_arrive(bar(C::bKVFull + slot));
                 }
+                // the row indices are in registers once the copies are issued: the list slot may be rebuilt
+                __syncwarp();
+                if (ok && lane == 0) mbar_arrive(bar(C::bListEmpty + ls));
             }
             cp_wait<0>();
             if (!ok) flag_status(a.status);
@@ -485,16 +514,8 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
                 const float off = m_run == -INFINITY ? 0.0f : w2 - m_run;
                 // P = 2^(s log2(e) + w2 - m_run); masked columns give 2^-inf = 0
                 uint32_t pk[32];
-                float l0 = 0.0f, l1 = 0.0f;
-#pragma unroll
-                for (int e = 0; e < 64; e += 2) {
-                    const float p0 = ex2_approx(fmaf(__uint_as_float(v[e]), kLog2e, off));
-                    const float p1 = ex2_approx(fmaf(__uint_as_float(v[e + 1]), kLog2e, off));
-                    l0 += p0;
-                    l1 += p1;
-                    pk[e / 2] = pack_bf16x2(p0, p1);
-                }
-                l = l * alpha + (l0 + l1);
+                const float ls = exp_half(v, off, pk);
+                l = l * alpha + ls;
                 // P_b is free: the score product of this chunk was issued after the P.V product that last read it
                 // (chunk k - 2), and its commit covered that product
                 tmem_st32(trow + C::kPCol + 64 * b + 32 * h, pk);
@@ -700,6 +721,7 @@ int launch_st_t(TcArgs args, int sms, cudaStream_t st) {
         args.items = args.lv.bh * args.lv.nodes * blocks * args.tiles_per_block;
         args.nb = args.lv.bp / kCK;
         args.ns = (args.m + kCK - 1) / kCK;
+        if (args.nb + args.ns > kMaxItemChunks) return -2;
     } else {
         args.per_outer = static_cast<uint32_t>(args.bh * args.nleaves);
         args.items = static_cast<int64_t>(args.tiles_per_leaf) * args.bh * args.nleaves;

@@ -26,7 +26,7 @@ EXPORTS = [
     "hyper_attn_status", "hyper_attn_last_launch_count", "hyper_attn_last_error", "hyper_attn_destroy",
     "hyper_attn_version", "hyper_attn_profile", "hyper_attn_profile_read",
     "hyper_attn_last_kernel", "hyper_attn_forward_noalloc", "hyper_attn_exact",
-    "hyper_attn_diagnostics", "hyper_attn_backward",
+    "hyper_attn_diagnostics", "hyper_attn_backward", "hyper_attn_test_fail_alloc",
 ]
 KERNEL_CLASSES = ["hash", "sort", "attn", "causal_base", "draws"]
 
@@ -73,6 +73,7 @@ def lib():
     L.hyper_attn_exact.argtypes = [vp, vp, vp, vp, vp, i64, ci, ci, ci]
     L.hyper_attn_diagnostics.argtypes = [vp, vp, vp, i64, ci, ci, ci, ci, u64, i64, vp, vp]
     L.hyper_attn_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i64, ci, ci, ci, ci, ci, ci, u64]
+    L.hyper_attn_test_fail_alloc.argtypes = [vp, ci]
     L.hyper_attn_draw.argtypes = [u64, ci, ci, i64, i64, ci, ci, i64, vp, vp]
     L.hyper_attn_levels.argtypes = [i64, ci, i64, ctypes.POINTER(ci), ctypes.POINTER(i64)]
     L.hyper_attn_debug_copy.argtypes = [vp, ci, ci, vp, ctypes.c_size_t]
@@ -197,6 +198,10 @@ class HyperAttention:
 
     def last_error(self) -> str:
         return lib().hyper_attn_last_error(self._h).decode()
+
+    def test_fail_alloc(self, count: int):
+        """Test hook: fail the handle's next `count` allocations as if memory had run out (HA_ERR_OOM)."""
+        self._check(lib().hyper_attn_test_fail_alloc(self._h, count))
 
     def profile(self, enable: bool):
         self._check(lib().hyper_attn_profile(self._h, int(enable)))

@@ -26,6 +26,8 @@ struct hyper_attn_s {
     size_t io_bytes = 0;
     cudaStream_t cs_in = nullptr, cs_out = nullptr;
     std::vector<cudaEvent_t> pipe_ev;
+    // test hook: the number of upcoming allocations to fail (hyper_attn_test_fail_alloc)
+    int fail_alloc = 0;
     // draws currently resident in the workspace
     bool draws_valid = false;
     uint64_t dk_seed = 0;
@@ -227,6 +229,23 @@ size_t plan_layout(const Shape &s, int esz_in, int capture, bool rownorm, hyper_
     return off;
 }
 
+// Every allocation of a handle goes through these, so that the allocation-failure test hook can fail one.
+cudaError_t device_alloc(hyper_attn_t h, unsigned char **p, size_t bytes) {
+    if (h->fail_alloc > 0) {
+        --h->fail_alloc;
+        return cudaErrorMemoryAllocation;
+    }
+    return cudaMalloc(p, bytes);
+}
+
+cudaError_t host_alloc(hyper_attn_t h, unsigned char **p, size_t bytes) {
+    if (h->fail_alloc > 0) {
+        --h->fail_alloc;
+        return cudaErrorMemoryAllocation;
+    }
+    return cudaMallocHost(p, bytes);
+}
+
 int ensure_workspace(hyper_attn_t h, size_t bytes) {
     if (bytes <= h->ws_bytes) return HA_OK;
     if (h->ws) {
@@ -238,7 +257,7 @@ int ensure_workspace(hyper_attn_t h, size_t bytes) {
     }
     h->draws_valid = false;
     const size_t want = align_up(bytes + bytes / 8, 1 << 20);
-    if (cudaMalloc(&h->ws, want) != cudaSuccess) {
+    if (device_alloc(h, &h->ws, want) != cudaSuccess) {
         cudaGetLastError();
         h->ws = nullptr;
         return fail(h, HA_ERR_OOM, "workspace allocation of %zu bytes failed", want);
@@ -257,7 +276,7 @@ int ensure_pinned(hyper_attn_t h, size_t bytes) {
         h->pin_bytes = 0;
     }
     const size_t want = align_up(bytes, 1 << 16);
-    if (cudaMallocHost(&h->pin, want) != cudaSuccess) {
+    if (host_alloc(h, &h->pin, want) != cudaSuccess) {
         cudaGetLastError();
         h->pin = nullptr;
         return fail(h, HA_ERR_OOM, "page-locked staging of %zu bytes failed", want);
@@ -715,7 +734,7 @@ int hyper_attn_forward_host(hyper_attn_t h, const void *Q, const void *K, const 
             h->io = nullptr;
             h->io_bytes = 0;
         }
-        if (cudaMalloc(&h->io, need) != cudaSuccess) {
+        if (device_alloc(h, &h->io, need) != cudaSuccess) {
             cudaGetLastError();
             h->io = nullptr;
             return fail(h, HA_ERR_OOM, "device buffers of %zu bytes failed", need);
@@ -875,6 +894,12 @@ int hyper_attn_last_kernel(hyper_attn_t h) { return h ? h->last_kernel : 0; }
 int hyper_attn_last_launch_count(hyper_attn_t h) { return h ? h->last_launches : 0; }
 
 const char *hyper_attn_last_error(hyper_attn_t h) { return h ? h->err.c_str() : "null handle"; }
+
+int hyper_attn_test_fail_alloc(hyper_attn_t h, int count) {
+    if (!h || count < 0) return HA_ERR_INVALID_ARG;
+    h->fail_alloc = count;
+    return HA_OK;
+}
 
 int hyper_attn_destroy(hyper_attn_t h) {
     if (!h) return HA_OK;

@@ -81,7 +81,7 @@ struct STCfg {
     static constexpr int bQFull = 0, bQEmpty = bQFull + QB, bKVFull = bQEmpty + QB, bKVEmpty = bKVFull + NST,
                          bWordFull = bKVEmpty + NST, bListFull = bWordFull + NST, bListEmpty = bListFull + 2,
                          bSFull = bListEmpty + 2,
-                         bPFull = bSFull + 2, bPVDone = bPFull + 2, bOReady = bPVDone + 2, bOFree = bOReady + 2,
+                         bPFull = bSFull + 2, bOReady = bPFull + 2, bOFree = bOReady + 2,
                          bStatsReady = bOFree + 2, bStatsFree = bStatsReady + 2, bDrain = bStatsFree + 2,
                          kNumBars = bDrain + 1;
     static constexpr int kTmemSlot = kBars + kNumBars * 8;
@@ -191,7 +191,6 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar(C::bSFull + b), 1);      // commit after a score product into S_b
             mbar_init(bar(C::bPFull + b), 256);    // both softmax warpgroups: their halves of P_b written
-            mbar_init(bar(C::bPVDone + b), 1);     // commit after the P.V product that read P_b
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar(C::bOReady + i), 1);     // commit after an item's last P.V product (item parity i)
@@ -435,7 +434,6 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
                     for (int kk = 0; kk < kCK / 16; ++kk)
                         mma_ts(od, tmem + C::kPCol + 64 * b + kk * 8, dv + static_cast<uint64_t>((kk * 2048) >> 4),
                                idesc_pv, (c > 0 || kk > 0) ? 1u : 0u);
-                    mma_commit(bar(C::bPVDone + b));
                     if (c == x.nc - 1) mma_commit(bar(C::bOReady + ip));
                     mma_commit(bar(C::bKVEmpty + slot));   // both products of chunk k have been issued
                     ok = issue_next_s();                   // chunk k + 2 into buffer k mod 2
@@ -520,10 +518,10 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
                 // (chunk k - 2), and its commit covered that product
                 tmem_st32(trow + C::kPCol + 64 * b + 32 * h, pk);
                 if (rescale) {
-                    // O holds the P.V products of the item's chunks before this one: wait for the last (chunk k - 1),
-                    // then scale this half's 32 of its columns
+                    // O holds the P.V products of the item's chunks before this one: wait for the last (chunk k - 1;
+                    // the commit that frees its K/V stage follows it), then scale this half's 32 of its columns
                     const uint32_t kp = k - 1;
-                    if (!mbar_wait_inl(bar(C::bPVDone + (kp & 1)), (kp >> 1) & 1, abort_flag)) ok = false;
+                    if (!mbar_wait_inl(bar(C::bKVEmpty + kp % C::NST), (kp / C::NST) & 1, abort_flag)) ok = false;
                     if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
                     tc_fence_after();
                     uint32_t o[32];

@@ -244,6 +244,13 @@ HA_API int hyper_attn_last_launch_count(hyper_attn_t h);
 /* Text of the last error on this handle ("" if none). Valid until the next call on the handle. */
 HA_API const char *hyper_attn_last_error(hyper_attn_t h);
 
+/* Test hook for the allocation-failure path: the handle's next `count` allocations (its device workspace, its
+ * page-locked staging buffer, the device copies of hyper_attn_forward_host) fail as if the device or the host
+ * had no memory left, without calling CUDA. The call that meets one returns HA_ERR_OOM before it enqueues any
+ * kernel or copy, the caller's buffers are left as they were, and the handle stays usable: the next call
+ * allocates again. count = 0 clears the hook. Returns HA_ERR_INVALID_ARG for a null handle or count < 0. */
+HA_API int hyper_attn_test_fail_alloc(hyper_attn_t h, int count);
+
 /* Release the workspace and the handle. NULL is accepted. Synchronises the handle's stream first. */
 HA_API int hyper_attn_destroy(hyper_attn_t h);
 

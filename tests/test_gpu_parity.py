@@ -117,6 +117,41 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_hash_planted_near_zero(ha, dtype):
+    """Rows planted on the near-zero boundary of the sortLSH signs ("HyperAttention: Long-context Attention in
+    Near-Linear Time", summary page, "Approach": bit j is the sign of x.P_j). fp32: every 4th query and key row
+    has its component along P_(row mod r) removed in float64, so that |x.P_j| lands far below 1e-4 * ||x||;
+    bf16 (whose rounding cannot get that close): every 16th row is exactly zero, the sign tie (bit 0, not
+    flagged). Ranks, flags, permutations and the output must match the oracle exactly like everywhere else."""
+    n, d, bh, block, m, r, seed = 4096, 64, 2, 256, 128, 8, 4242
+    Qh, Kh, Vh = wl.make_inputs(n, d, bh, data_seed=77, planted=0.05, dtype=dtype)
+    P = oracle.draw_projection(seed, d, r).astype(np.float64)
+    if dtype == "fp32":
+        for X in (Qh, Kh):
+            rows = np.arange(0, n, 4)
+            for h in range(bh):
+                x = X[h, rows].astype(np.float64)
+                pj = P[:, rows % r].T                                   # (rows, d): the projection each row loses
+                x -= ((x * pj).sum(axis=1) / (pj * pj).sum(axis=1))[:, None] * pj
+                X[h, rows] = x.astype(np.float32)
+    else:
+        for X in (Qh, Kh):
+            X[:, ::16] = 0
+    Qf, Kf, Vf = wl.as_f32(Qh), wl.as_f32(Kh), wl.as_f32(Vh)
+    got = run_gpu(ha, Qh, Kh, Vh, n=n, d=d, bh=bh, block=block, m=m, r=r, causal=False, seed=seed, dtype=dtype,
+                  kernel="auto")
+    check_ranks_and_perms(ha, Qf, Kf, n=n, bh=bh, r=r, causal=False, base=4096, seed=seed)
+    near = ha.debug_copy("near", 0, np.uint8, bh * 2 * n).reshape(bh, 2, n)
+    if dtype == "fp32":
+        assert near[:, :, ::4].mean() > 0.99, "planted rows are flagged near zero"
+    else:
+        assert not near[:, :, ::16].any(), "zero rows: every projection is exactly 0, which is not below 0"
+    for h in range(bh):
+        ref = oracle.forward(Qf[h], Kf[h], Vf[h], block=block, m=m, r=r, causal=False, seed=seed, bh=h)
+        assert rel_err(got[h], ref["O"]) < TOL[dtype]
+
+
 @pytest.mark.parametrize("kernel", ["simt", "auto", "tc"])
 @pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
 def test_parity_small(ha, case, kernel):

@@ -73,13 +73,12 @@ struct STCfg {
     static constexpr int kKPerm = kCacheB + kMaxSampleList * 4;           // key rows of the current block
     static constexpr int kQPerm = kKPerm + kMaxBlock * 4;                 // query rows of one tile
     static constexpr int kIList = kQPerm + 128 * 4;                       // [item parity]: global key rows per chunk
-    static constexpr int kIWord = kIList + 2 * kMaxItemChunks * kCK * 4;  // [item parity]: valid columns per chunk
-    static constexpr int kStats = kIWord + 2 * kMaxItemChunks * 4;        // [item parity][half][row]: max, sum
+    static constexpr int kICnt = kIList + 2 * kMaxItemChunks * kCK * 4;   // [item parity]: kept samples of the item
+    static constexpr int kStats = kICnt + 16;                             // [item parity][half][row]: max, sum
     static constexpr int kXch = kStats + 2 * 2 * 128 * 8;                 // [chunk parity][half][row]: partial maxima
-    static constexpr int kWord = kXch + 2 * 2 * 128 * 4;
-    static constexpr int kBars = (kWord + NST * 4 + 15) / 16 * 16;
+    static constexpr int kBars = kXch + 2 * 2 * 128 * 4;
     static constexpr int bQFull = 0, bQEmpty = bQFull + QB, bKVFull = bQEmpty + QB, bKVEmpty = bKVFull + NST,
-                         bWordFull = bKVEmpty + NST, bListFull = bWordFull + NST, bListEmpty = bListFull + 2,
+                         bListFull = bKVEmpty + NST, bListEmpty = bListFull + 2,
                          bSFull = bListEmpty + 2,
                          bPFull = bSFull + 2, bOReady = bPFull + 2, bOFree = bOReady + 2,
                          bStatsReady = bOFree + 2, bStatsFree = bStatsReady + 2, bDrain = bStatsFree + 2,
@@ -169,7 +168,7 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
     const uint32_t sbase = raw_addr + pad;
     auto bar = [&](int i) -> uint32_t { return sbase + C::kBars + 8u * static_cast<uint32_t>(i); };
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + C::kAbort);
-    int *words = reinterpret_cast<int *>(sm + C::kWord);
+    int *icnt = reinterpret_cast<int *>(sm + C::kICnt);
     float2 *stats = reinterpret_cast<float2 *>(sm + C::kStats);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -182,11 +181,10 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
         for (int s = 0; s < C::NST; ++s) {
             mbar_init(bar(C::bKVFull + s), 64);    // the K and V loader warps' lanes (copy completion)
             mbar_init(bar(C::bKVEmpty + s), 1);    // commit after the chunk's P.V product
-            mbar_init(bar(C::bWordFull + s), 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar(C::bListFull + i), 1);   // the list builder: an item's key rows and column counts written
-            mbar_init(bar(C::bListEmpty + i), 2);  // the K and V loaders: done with the item's list
+            mbar_init(bar(C::bListEmpty + i), 10); // the K and V loaders and the 8 softmax warps: done with the list
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar(C::bSFull + b), 1);      // commit after a score product into S_b
@@ -253,7 +251,6 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
                     break;
                 }
                 int32_t *ilist = reinterpret_cast<int32_t *>(sm + C::kIList) + ls * (kMaxItemChunks * kCK);
-                int32_t *iword = reinterpret_cast<int32_t *>(sm + C::kIWord) + ls * kMaxItemChunks;
                 int64_t kbase = 0;
                 if (is_level(MODE)) {
                     kbase = static_cast<int64_t>(x.bhi) * a.n + static_cast<int64_t>(x.node) * a.lv.node_len;
@@ -295,7 +292,6 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
                 for (int c = 0; c < x.nc; ++c) {
                     const bool sample = is_level(MODE) && c < a.ns;
                     const int u0 = c * kCK;
-                    if (lane == 0) iword[c] = sample ? min(kCK, max(0, cnt - u0)) : kCK;
                     const int64_t cbase = is_level(MODE) ? kbase : x.leaf_start + static_cast<int64_t>(c) * kCK;
 #pragma unroll
                     for (int rr = 0; rr < kCK / 32; ++rr) {
@@ -307,6 +303,7 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
                         ilist[c * kCK + row] = static_cast<int32_t>(cbase + loc);
                     }
                 }
+                if (lane == 0) icnt[ls] = is_level(MODE) ? cnt : 0;
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(C::bListFull + ls));
                 // the query tile
@@ -336,8 +333,7 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
         } else if (warp == 0 || warp == 3) {
             // -------------------------------------------------------------- K loader (warp 0), V loader (warp 3)
             // chunk g of the CTA (over all items) goes to stage g mod NST once the stage's previous chunk has
-            // completed its products; rows from the item's list. The K loader also publishes the chunk's valid
-            // column count for the softmax.
+            // completed its products; rows from the item's list.
             const bool is_k = warp == 0;
             const uint16_t *src = is_k ? a.K : a.V;
             const uint32_t dst0 = sbase + (is_k ? C::kK : C::kV);
@@ -348,17 +344,12 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
                 const int ls = static_cast<int>(ni & 1);
                 if (!mbar_wait_inl(bar(C::bListFull + ls), (ni >> 1) & 1, abort_flag)) { ok = false; break; }
                 const int32_t *ilist = reinterpret_cast<const int32_t *>(sm + C::kIList) + ls * (kMaxItemChunks * kCK);
-                const int32_t *iword = reinterpret_cast<const int32_t *>(sm + C::kIWord) + ls * kMaxItemChunks;
                 for (int c = 0; c < x.nc; ++c, ++g) {
                     const int slot = static_cast<int>(g % C::NST);
                     const uint32_t round = g / C::NST;
                     if (round > 0 && !mbar_wait_inl(bar(C::bKVEmpty + slot), (round - 1) & 1, abort_flag)) {
                         ok = false;
                         break;
-                    }
-                    if (is_k && lane == 0) {
-                        words[slot] = iword[c];
-                        mbar_arrive(bar(C::bWordFull + slot));
                     }
                     gather_rows<D, true, kCK>(dst0 + slot * C::kCBytes, src, 0, ilist + c * kCK, lane);
                     cp_async_arrive(bar(C::bKVFull + slot));
@@ -460,6 +451,16 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
             const int ip = static_cast<int>(ni & 1);
             const uint32_t tO = trow + C::kOCol + D * ip + 32 * h;   // this half's share of the row's accumulator
             float m_run = -INFINITY, l = 0.0f;       // running max (base 2, weight included) and this half's sum
+            // the item's count of kept samples (the valid columns of its sample chunks), from its list slot
+            int cnt = 0;
+            if (is_level(MODE)) {
+                const int ls = static_cast<int>(ni & 1);
+                if (!mbar_wait_inl(bar(C::bListFull + ls), (ni >> 1) & 1, abort_flag)) ok = false;
+                if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
+                cnt = icnt[ls];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(C::bListEmpty + ls));
+            }
             for (int c = 0; c < x.nc; ++c, ++k) {
                 const int b = static_cast<int>(k & 1);
                 if (!mbar_wait_inl(bar(C::bSFull + b), (k >> 1) & 1, abort_flag)) { ok = false; break; }
@@ -468,9 +469,7 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
                 float w2 = 0.0f;
                 if (is_level(MODE)) {
                     if (c < a.ns) {
-                        const int slot = static_cast<int>(k % C::NST);
-                        if (!mbar_wait_inl(bar(C::bWordFull + slot), (k / C::NST) & 1, abort_flag)) { ok = false; break; }
-                        bound = words[slot] - 1;
+                        bound = min(kCK, max(0, cnt - c * kCK)) - 1;
                         w2 = a.lw2;
                     }
                 } else if (MODE == MODE_CAUSAL) {

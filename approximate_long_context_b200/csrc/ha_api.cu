@@ -28,8 +28,10 @@ struct hyper_attn_s {
     std::vector<cudaEvent_t> pipe_ev;
     // test hook: the number of upcoming allocations to fail (hyper_attn_test_fail_alloc)
     int fail_alloc = 0;
-    // draws currently resident in the workspace
+    // draws currently resident in the workspace, and a host copy of their projection matrix ([d][r]), which the
+    // hash kernel takes as launch parameters
     bool draws_valid = false;
+    std::vector<float> hostP;
     uint64_t dk_seed = 0;
     int dk_d = 0, dk_r = 0, dk_m = 0, dk_causal = 0;
     int64_t dk_bh = 0, dk_n = 0, dk_base = 0, dk_off = 0;
@@ -320,6 +322,7 @@ int upload_draws(hyper_attn_t h, uint64_t seed, const Shape &s, int64_t bh_offse
     float *P = reinterpret_cast<float *>(h->pin);
     int32_t *S = reinterpret_cast<int32_t *>(h->pin + pbytes);
     if (host_draws(seed, s, bh_offset, P, S)) return fail(h, HA_ERR_INVALID_ARG, "sample draw failed");
+    h->hostP.assign(P, P + static_cast<size_t>(s.d) * s.r);
     HA_CUDA(h, cudaMemcpyAsync(h->ws + h->lay.P, P, sizeof(float) * s.d * (s.r ? s.r : 1), cudaMemcpyHostToDevice, st));
     if (sbytes) HA_CUDA(h, cudaMemcpyAsync(h->ws + h->lay.S, S, sbytes, cudaMemcpyHostToDevice, st));
     HA_CUDA(h, cudaEventRecord(h->pin_free, st));
@@ -359,7 +362,6 @@ int run_forward(hyper_attn_t h, const void *Q, const void *K, const void *V, voi
     if (rc) return rc;
 
     unsigned char *ws = h->ws;
-    const float *P = reinterpret_cast<const float *>(ws + lay.P);
     const int32_t *S = reinterpret_cast<const int32_t *>(ws + lay.S);
     uint16_t *rank = reinterpret_cast<uint16_t *>(ws + lay.rank);
     uint8_t *near = ws + lay.near;
@@ -421,7 +423,7 @@ int run_forward(hyper_attn_t h, const void *Q, const void *K, const void *V, voi
         lwrn = rlw;
     }
     ev = prof_begin();
-    kl = ha::launch_hash(Q, K, dtype, s.bh, s.n, s.d, P, s.r, rank, near, st);
+    kl = ha::launch_hash(Q, K, dtype, s.bh, s.n, s.d, h->hostP.data(), s.r, rank, near, st);
     prof_end(ev, HA_KC_HASH, kl);
     if ((rc = count(kl, "hash"))) return rc;
 

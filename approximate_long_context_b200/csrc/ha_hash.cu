@@ -12,9 +12,9 @@
 // Layout: persistent CTAs of 128 threads walk tiles of 128 x RPT consecutive rows of the combined index
 // g = ((bh*2 + which)*n + row) (which 0 = Q, 1 = K), RPT rows per thread. Tiles are double-buffered in
 // shared memory: the 16-byte cp.async copies of tile i+1 (coalesced; row stride padded by 16 bytes against
-// bank conflicts) are in flight while tile i is hashed. P sits in shared memory as [d][r4] (r rounded up to
-// a multiple of 4); for each k a thread reads P[k][0..r) with broadcast 16-byte loads and advances each
-// projection's chain by one fused multiply-add.
+// bank conflicts) are in flight while tile i is hashed. P travels as a kernel parameter ([d][r4], r rounded
+// up to a multiple of 4): the loops over k and j are unrolled, so every fused multiply-add takes its P[k][j]
+// straight from the constant bank, with no load instruction.
 #include "ha_common.cuh"
 #include "ha_internal.h"
 
@@ -23,12 +23,18 @@ namespace {
 
 constexpr int kThreads = 128;
 
+// The projection matrix, [D][R4] (columns j >= r are zero).
+template <int D, int R4>
+struct HashProj {
+    float v[D * (R4 > 0 ? R4 : 1)];
+};
+
 // RPT rows per thread: a tile is kThreads * RPT consecutive rows; thread i hashes rows i, i + kThreads, ...
-// Each broadcast load of P then feeds RPT rows' fused multiply-adds.
 template <int D, int DTYPE, int R4, int RPT>
 __global__ void __launch_bounds__(kThreads) hash_kernel(const void *__restrict__ Q, const void *__restrict__ K,
-                                                        int64_t n, int64_t total_rows, const float *__restrict__ P,
-                                                        int r, uint16_t *__restrict__ rank, uint8_t *__restrict__ near) {
+                                                        int64_t n, int64_t total_rows,
+                                                        const __grid_constant__ HashProj<D, R4> P, int r,
+                                                        uint16_t *__restrict__ rank, uint8_t *__restrict__ near) {
     constexpr int kRows = kThreads * RPT;
     constexpr int ESZ = DTYPE == 0 ? 2 : 4;
     constexpr int ROW_BYTES = D * ESZ;
@@ -38,15 +44,9 @@ __global__ void __launch_bounds__(kThreads) hash_kernel(const void *__restrict__
     // R4: r rounded up to a multiple of 4 (compile time, so the unrolled loops carry no conditions); the
     // padded projections multiply zero columns of P and are ignored.
     extern __shared__ __align__(16) unsigned char smem[];
-    float *Ps = reinterpret_cast<float *>(smem);                               // [D][max(R4, 4)]
-    constexpr int PS = R4 > 0 ? R4 : 4;
-    unsigned char *tiles = smem + D * PS * sizeof(float);                      // [2][kRows][STRIDE]
+    unsigned char *tiles = smem;                                               // [2][kRows][STRIDE]
 
     const int tid = threadIdx.x;
-    for (int i = tid; i < D * PS; i += kThreads) {
-        const int k = i / PS, j = i % PS;
-        Ps[i] = j < r ? P[k * r + j] : 0.0f;
-    }
     const int64_t ntiles = (total_rows + kRows - 1) / kRows;
 
     // stage one tile with 16-byte copies. A tile inside one segment (the usual case) is kRows * ROW_BYTES
@@ -89,7 +89,7 @@ __global__ void __launch_bounds__(kThreads) hash_kernel(const void *__restrict__
         } else {
             cp_async_wait<0>();
         }
-        __syncthreads();   // tile `buf` (and P on the first pass) visible to every thread
+        __syncthreads();   // tile `buf` visible to every thread
 
         const unsigned char *rows = tiles + buf * (kRows * STRIDE) + tid * STRIDE;
         float acc[RPT][R4 > 0 ? R4 : 1];
@@ -100,7 +100,7 @@ __global__ void __launch_bounds__(kThreads) hash_kernel(const void *__restrict__
 #pragma unroll
             for (int j = 0; j < R4; ++j) acc[q][j] = 0.0f;
         }
-#pragma unroll 2
+#pragma unroll
         for (int c = 0; c < CHUNKS; ++c) {
             float x[RPT][EPC];
 #pragma unroll
@@ -125,17 +125,11 @@ __global__ void __launch_bounds__(kThreads) hash_kernel(const void *__restrict__
                 const int k = c * EPC + e;
 #pragma unroll
                 for (int q = 0; q < RPT; ++q) nrm2[q] = __fmaf_rn(x[q][e], x[q][e], nrm2[q]);
-                const float4 *pk = reinterpret_cast<const float4 *>(Ps + k * PS);
 #pragma unroll
-                for (int q4 = 0; q4 < R4 / 4; ++q4) {
-                    const float4 p = pk[q4];
+                for (int j = 0; j < R4; ++j) {
+                    const float p = P.v[k * R4 + j];
 #pragma unroll
-                    for (int q = 0; q < RPT; ++q) {
-                        acc[q][4 * q4 + 0] = __fmaf_rn(x[q][e], p.x, acc[q][4 * q4 + 0]);
-                        acc[q][4 * q4 + 1] = __fmaf_rn(x[q][e], p.y, acc[q][4 * q4 + 1]);
-                        acc[q][4 * q4 + 2] = __fmaf_rn(x[q][e], p.z, acc[q][4 * q4 + 2]);
-                        acc[q][4 * q4 + 3] = __fmaf_rn(x[q][e], p.w, acc[q][4 * q4 + 3]);
-                    }
+                    for (int q = 0; q < RPT; ++q) acc[q][j] = __fmaf_rn(x[q][e], p, acc[q][j]);
                 }
             }
         }
@@ -175,11 +169,14 @@ int num_sms_hash() {
 template <int D, int DTYPE, int R4>
 int launch_hash_t(const void *Q, const void *K, int64_t bh, int64_t n, const float *P, int r, uint16_t *rank,
                   uint8_t *near, cudaStream_t st) {
+    HashProj<D, R4> proj{};
+    for (int k = 0; k < D; ++k)
+        for (int j = 0; j < r; ++j) proj.v[k * R4 + j] = P[k * r + j];
     constexpr int ESZ = DTYPE == 0 ? 2 : 4;
     // two rows per thread while a double-buffered tile stays small (rows of up to 256 bytes)
     constexpr int RPT = D * ESZ <= 256 ? 2 : 1;
     constexpr int kRows = kThreads * RPT;
-    const size_t smem = D * (R4 > 0 ? R4 : 4) * sizeof(float) + 2 * kRows * (D * ESZ + 16);
+    const size_t smem = 2 * kRows * (D * ESZ + 16);
     auto kern = hash_kernel<D, DTYPE, R4, RPT>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
         return -1;
@@ -190,7 +187,7 @@ int launch_hash_t(const void *Q, const void *K, int64_t bh, int64_t n, const flo
     const int64_t ntiles = (total + kRows - 1) / kRows;
     const int64_t slots = static_cast<int64_t>(num_sms_hash()) * per_sm;
     const int64_t grid = ntiles < slots ? ntiles : slots;
-    kern<<<static_cast<unsigned>(grid), kThreads, smem, st>>>(Q, K, n, total, P, r, rank, near);
+    kern<<<static_cast<unsigned>(grid), kThreads, smem, st>>>(Q, K, n, total, proj, r, rank, near);
     return cudaPeekAtLastError() == cudaSuccess ? 1 : -1;
 }
 
@@ -208,7 +205,7 @@ int launch_hash_r(const void *Q, const void *K, int64_t bh, int64_t n, const flo
 
 }  // namespace
 
-// P: [d][r] float in device memory.
+// P: [d][r] float in host memory (copied into the launch's parameters).
 int launch_hash(const void *Q, const void *K, int dtype, int64_t bh, int64_t n, int d, const float *P, int r,
                 uint16_t *rank, uint8_t *near, cudaStream_t st) {
     if (r < 0 || r > kMaxR || (d != 64 && d != 128)) return -1;

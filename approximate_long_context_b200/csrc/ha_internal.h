@@ -38,7 +38,7 @@ struct SortPass {
 // ---- kernels (launch wrappers return the number of kernels launched, or -1 on launch error) ----
 
 // sortLSH hash of 2*bh*n rows (Q rows then K rows of each problem): rank[bh][2][n], near[bh][2][n].
-// P is the [d][r] projection matrix in device memory.
+// P is the [d][r] projection matrix in host memory (it travels in the launch's parameters).
 int launch_hash(const void *Q, const void *K, int dtype, int64_t bh, int64_t n, int d, const float *P, int r,
                 uint16_t *rank, uint8_t *near, cudaStream_t st);
 

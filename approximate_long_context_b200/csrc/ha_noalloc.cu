@@ -101,7 +101,6 @@ extern "C" int hyper_attn_forward_noalloc(const void *Q, const void *K, const vo
     ha::Level lv{};
     lv.n = n; lv.bh = heads; lv.level = 0; lv.nodes = 1; lv.node_len = n; lv.seg_len = n; lv.q_off = 0;
     lv.heap0 = 1; lv.bp = static_cast<int>(bp);
-    const float *P = reinterpret_cast<const float *>(base + kPOff);
     const int32_t *S = reinterpret_cast<const int32_t *>(base + kSOff);
     uint16_t *rank = reinterpret_cast<uint16_t *>(base + kRankOff);
     uint8_t *near = base + kNearOff;
@@ -111,7 +110,7 @@ extern "C" int hyper_attn_forward_noalloc(const void *Q, const void *K, const vo
 
     // a failed launch leaves its error behind: take it, so that the caller's next check starts clean
     const ha::SortPass pass{0, 1 << r};
-    if (ha::launch_hash(Q, K, dtype, heads, n, d, P, r, rank, near, st) < 0 ||
+    if (ha::launch_hash(Q, K, dtype, heads, n, d, g_P, r, rank, near, st) < 0 ||
         ha::launch_sort_pass(lv, rank, pass, nullptr, hist, perm, inv, st) < 0 ||
         ha::launch_attn_simt(lv, Q, K, V, dtype, d, perm, inv, S, m, 1, O, dtype, nullptr, nullptr, nullptr, st) < 0) {
         cudaGetLastError();

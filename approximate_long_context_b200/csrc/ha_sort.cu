@@ -10,10 +10,10 @@
 //   count   -- per 2048-row chunk of a segment, a shared-memory histogram of the digit;
 //   scan    -- per segment, turn the chunk histograms into the first output position of every
 //              (chunk, digit) pair (digit-major, chunks in order);
-//   scatter -- per chunk, 8 warps each own a contiguous 256-row slice; a warp ranks equal digits inside a
-//              32-row step with __match_any_sync and keeps running per-digit counters, so rows leave in
-//              their original order within each digit. The chunk is ordered in shared memory first, so
-//              that the permutation is written in runs of consecutive slots.
+//   scatter -- per chunk, 8 warps each own a contiguous 256-row slice; a warp finds the rows of equal digit
+//              inside a 32-row step with one ballot per digit bit and keeps running per-digit counters, so
+//              rows leave in their original order within each digit. The chunk is ordered in shared memory
+//              first, so that the permutation is written in runs of consecutive slots.
 // No kernel waits on another CTA: the three launches replace a look-back scan.
 #include "ha_common.cuh"
 #include "ha_internal.h"
@@ -148,7 +148,8 @@ __device__ __forceinline__ void block_exclusive_scan(int *a, int R, int *warp_su
 // order and its global position (the digit's first slot for this chunk, from the scan, plus its rank among
 // the chunk's rows of that digit). The inverse permutation is written in row order; the permutation is
 // written from the digit-sorted order, so that rows of one digit land in consecutive slots.
-__global__ void __launch_bounds__(kSortWarps * 32) sort_scatter_kernel(Level lv, const uint16_t *__restrict__ rank,
+template <int NBITS>   // log2 of the radix
+__global__ void __launch_bounds__(kSortWarps * 32, 4) sort_scatter_kernel(Level lv, const uint16_t *__restrict__ rank,
                                                                        SortPass ps, const int32_t *__restrict__ in_idx,
                                                                        const int32_t *__restrict__ hist, int cps,
                                                                        int32_t *__restrict__ perm,
@@ -165,13 +166,18 @@ __global__ void __launch_bounds__(kSortWarps * 32) sort_scatter_kernel(Level lv,
     const int c = blockIdx.x % cps;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const unsigned lt_mask = (1u << lane) - 1u;
-    for (int i = threadIdx.x; i < kSortWarps * R; i += blockDim.x) wcnt[i] = 0;
-    __syncthreads();
-
     const SegView v = seg_view(lv, rank, s);
     const int64_t start = static_cast<int64_t>(c) * kSortChunk;
     const int64_t end = min(lv.seg_len, start + kSortChunk);
     constexpr int kSlice = kSortChunk / kSortWarps;
+    // this chunk's first global slot of each digit (from the scan), loaded early (R <= 4 * blockDim)
+    const int32_t *h = hist + (s * cps + c) * R;
+    int gb_pref[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int b = threadIdx.x + u * kSortWarps * 32;
+        gb_pref[u] = b < R ? h[b] : 0;
+    }
     const int64_t lo = min(end, start + static_cast<int64_t>(warp) * kSlice);
     const int64_t hi = min(end, lo + kSlice);
     int *mycnt = wcnt + warp * R;
@@ -187,10 +193,20 @@ __global__ void __launch_bounds__(kSortWarps * 32) sort_scatter_kernel(Level lv,
         rowv[i] = 0;
         keyv[i] = p < hi ? digit_of(v, in_idx, p, ps, rowv[i]) : -1;
     }
+    for (int i = threadIdx.x; i < kSortWarps * R; i += blockDim.x) wcnt[i] = 0;
+    __syncthreads();
 #pragma unroll
     for (int i = 0; i < STEPS; ++i) {
         const int key = keyv[i];
-        const unsigned peers = __match_any_sync(0xffffffffu, key);
+        // the lanes holding the same key: one ballot for validity, one per digit bit
+        unsigned peers = __ballot_sync(0xffffffffu, key >= 0);
+        if (key < 0) peers = ~peers;
+#pragma unroll
+        for (int bb = 0; bb < NBITS; ++bb) {
+            const bool bit = (key >> bb) & 1;
+            const unsigned bal = __ballot_sync(0xffffffffu, bit);
+            peers &= bit ? bal : ~bal;
+        }
         const int before = key >= 0 ? mycnt[key] : 0;
         __syncwarp();
         if (key >= 0 && lane == __ffs(peers) - 1) mycnt[key] = before + __popc(peers);
@@ -198,12 +214,15 @@ __global__ void __launch_bounds__(kSortWarps * 32) sort_scatter_kernel(Level lv,
         rk[i] = before + __popc(peers & lt_mask);
     }
     __syncthreads();
-    const int32_t *h = hist + (s * cps + c) * R;
-    for (int b = threadIdx.x; b < R; b += blockDim.x) {
-        int tot = 0;
-        for (int w = 0; w < kSortWarps; ++w) tot += wcnt[w * R + b];
-        coff[b] = tot;
-        gbase[b] = h[b];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int b = threadIdx.x + u * kSortWarps * 32;
+        if (b < R) {
+            int tot = 0;
+            for (int w = 0; w < kSortWarps; ++w) tot += wcnt[w * R + b];
+            coff[b] = tot;
+            gbase[b] = gb_pref[u];
+        }
     }
     __syncthreads();
     block_exclusive_scan(coff, R, wsum);
@@ -232,6 +251,17 @@ __global__ void __launch_bounds__(kSortWarps * 32) sort_scatter_kernel(Level lv,
     for (int lp = threadIdx.x; lp < nloc; lp += blockDim.x) perm[v.out + sgpos[lp]] = srow[lp];
 }
 
+template <int NBITS>
+bool launch_scatter(int64_t grid, size_t smem, cudaStream_t st, const Level &lv, const uint16_t *rank, SortPass ps,
+                    const int32_t *in_idx, const int32_t *hist, int cps, int32_t *perm, int32_t *inv) {
+    auto kern = sort_scatter_kernel<NBITS>;
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+        return false;
+    kern<<<static_cast<unsigned>(grid), kSortWarps * 32, smem, st>>>(lv, rank, ps, in_idx, hist, cps, perm, inv);
+    return true;
+}
+
 }  // namespace
 
 int launch_sort_pass(const Level &lv, const uint16_t *rank, SortPass ps, const int32_t *in_idx, int32_t *hist,
@@ -243,12 +273,23 @@ int launch_sort_pass(const Level &lv, const uint16_t *rank, SortPass ps, const i
     sort_count_kernel<<<static_cast<unsigned>(grid), 256, ps.radix * sizeof(int), st>>>(lv, rank, ps, in_idx, hist, cps);
     sort_scan_kernel<<<static_cast<unsigned>(nseg), 1024, 0, st>>>(ps.radix, cps, hist);
     const size_t smem = (static_cast<size_t>(kSortWarps + 2) * ps.radix + kSortWarps + 2 * kSortChunk) * sizeof(int);
-    if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(sort_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
-            cudaSuccess)
-        return -1;
-    sort_scatter_kernel<<<static_cast<unsigned>(grid), kSortWarps * 32, smem, st>>>(lv, rank, ps, in_idx, hist, cps,
-                                                                                    perm, inv);
+    int nbits = 0;
+    while ((1 << nbits) < ps.radix) ++nbits;
+    int ok = 0;
+    switch (nbits) {
+        case 0: ok = launch_scatter<0>(grid, smem, st, lv, rank, ps, in_idx, hist, cps, perm, inv); break;
+        case 1: ok = launch_scatter<1>(grid, smem, st, lv, rank, ps, in_idx, hist, cps, perm, inv); break;
+        case 2: ok = launch_scatter<2>(grid, smem, st, lv, rank, ps, in_idx, hist, cps, perm, inv); break;
+        case 3: ok = launch_scatter<3>(grid, smem, st, lv, rank, ps, in_idx, hist, cps, perm, inv); break;
+        case 4: ok = launch_scatter<4>(grid, smem, st, lv, rank, ps, in_idx, hist, cps, perm, inv); break;
+        case 5: ok = launch_scatter<5>(grid, smem, st, lv, rank, ps, in_idx, hist, cps, perm, inv); break;
+        case 6: ok = launch_scatter<6>(grid, smem, st, lv, rank, ps, in_idx, hist, cps, perm, inv); break;
+        case 7: ok = launch_scatter<7>(grid, smem, st, lv, rank, ps, in_idx, hist, cps, perm, inv); break;
+        case 8: ok = launch_scatter<8>(grid, smem, st, lv, rank, ps, in_idx, hist, cps, perm, inv); break;
+        case 9: ok = launch_scatter<9>(grid, smem, st, lv, rank, ps, in_idx, hist, cps, perm, inv); break;
+        default: ok = launch_scatter<10>(grid, smem, st, lv, rank, ps, in_idx, hist, cps, perm, inv); break;
+    }
+    if (!ok) return -1;
     return cudaPeekAtLastError() == cudaSuccess ? 3 : -1;
 }
 

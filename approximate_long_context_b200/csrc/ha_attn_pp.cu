@@ -1,5 +1,6 @@
-// ha_attn_pp.cu -- tensor-core (tcgen05 / TMEM) attention for d = 64: one 128-query tile per CTA, double-buffered
-// score and probability tiles, two softmax warpgroups on the two column halves of every chunk.
+// ha_attn_pp.cu -- tensor-core (tcgen05 / TMEM) attention of the levels (block and sampled columns, merged), for
+// d = 64 and d = 128: one 128-query tile per work item, double-buffered score and probability tiles, two softmax
+// warpgroups on the two column halves of every chunk.
 //
 // The work is the same as in ha_attn_tc.cu ("HyperAttention: Long-context Attention in Near-Linear Time",
 // research-map summary, "Approach"): the queries of a sorted block attend exactly to the block's keys and, with the
@@ -15,28 +16,34 @@
 //   * The exponentials (MUFU unit, 16 per clock per SM) bound the softmax. Two warpgroups share every chunk: warp w
 //     handles rows 32 (w mod 4) .. 32 (w mod 4) + 31 and column half h = (w - 4) / 4, so each sub-partition runs two
 //     softmax warps. The halves of a row exchange their partial maxima through shared memory (a 64-thread named
-//     barrier per lane quarter) and keep partial sums, which the epilogue adds.
+//     barrier per lane quarter) and keep partial sums, which the epilogue adds. The exponent's scale and offset and
+//     the row sums run as packed f32x2 instructions.
 //   * The MMA issuer, per chunk k: wait for P(k), issue O += P(k) V(k), then the score product of chunk k + 2 into
 //     the buffer that chunk k has just released; each commit of a score product therefore also covers the P.V
 //     product of two chunks back, so a P buffer is always free when its next scores arrive. A row is re-based only
 //     when its max grows by more than 2^8; O is then scaled after the previous chunk's P.V product has completed.
+//   * One warp builds, an item ahead, the global key rows of every chunk of the item (through the key permutation,
+//     and the sampled columns whose key lies outside the block, compacted) and the item's count of kept samples;
+//     the K and V loaders then only copy rows, and the softmax takes its masking from the count.
 //   * A warpgroup of its own runs the epilogue (normalise, write each row to its original position, or write a causal
-//     level's part). The accumulator is double-buffered by item, and the epilogue reads it into registers and releases
-//     it before it writes, so the next item's first P.V product never waits on it.
+//     level's part). d = 64: the accumulator is double-buffered by item, and the epilogue reads it into registers and
+//     releases it before it writes, so the next item's first P.V product never waits on it. d = 128: one accumulator
+//     (TMEM holds no second one), released once the epilogue has read the row.
 //
 // CTA layout (512 threads, one CTA per SM, persistent):
-//   warp 0       K loader (rows through the key permutation or the compacted sample list),
+//   warp 0       K loader,
 //   warp 1       MMA issuer (lane 0),
-//   warp 2       Q loader,
+//   warp 2       row-list builder and Q loader,
 //   warp 3       V loader,
 //   warps 4-7    softmax of column half 0, warps 8-11 softmax of column half 1 (warp w reads TMEM lanes
 //                32 (w mod 4) .. 32 (w mod 4) + 31),
 //   warps 12-15  epilogue.
 // Loaders copy rows with 16-byte cp.async into the 128-byte-swizzled layout the tensor core reads and arrive on the
-// stage barrier when their copies complete. Registers per thread: softmax kRegsSoftmax, the others kRegsOther
-// (4 x 128 threads x 128 at launch).
-// TMEM (512 columns): S_b at [128 b, 128 b + 128), P_b at [256 + 64 b, ...) (column half h at + 32 h), O of items of
-// parity i at [384 + 64 i, ...) (b, i = 0, 1).
+// stage's K or V barrier when their copies complete. Stages: 4 (d = 64) or 2 (d = 128); with two, a K stage is
+// refilled as soon as its chunk's score product has completed, a V stage once its P.V product has. Registers per
+// thread: softmax kRegsSoftmax, the others kRegsOther (4 x 128 threads x 128 at launch).
+// TMEM (512 columns): S_b at [128 b, 128 b + 128), P_b at [256 + 64 b, ...) (column half h at + 32 h), O accumulator j
+// at [384 + d j, 384 + d (j + 1)) (b = 0, 1; j < 2 for d = 64, j = 0 for d = 128).
 // Every mbarrier wait is bounded; on expiry the kernel sets the status bit, every role gives up, the loaders wait for
 // their copies, the MMA issuer drains the tensor core, and TMEM is freed before exit.
 #include "ha_attn_items.cuh"
@@ -55,14 +62,16 @@ static_assert(128 * (2 * kRegsSoftmax + 2 * kRegsOther) == kSTThreads * 128,
 constexpr int kCK = 128;            // keys per chunk
 constexpr int kMaxItemChunks = kMaxBlock / kCK + kMaxSampleList / kCK;   // block chunks + sample chunks of an item
 
+template <int D_>
 struct STCfg {
-    static constexpr int D = 64;
-    static constexpr int QB = 2;                       // Q buffers
-    static constexpr int NST = 4;                      // K/V stages of kCK rows
+    static constexpr int D = D_;
+    static constexpr int QB = D == 64 ? 2 : 1;         // Q buffers
+    static constexpr int NST = D == 64 ? 4 : 2;        // K/V stages of kCK rows
+    static constexpr int OB = D == 64 ? 2 : 1;         // O accumulators (item i uses i mod OB)
     static constexpr int kQBytes = 128 * D * 2;        // a Q tile
     static constexpr int kCBytes = kCK * D * 2;        // a K or V chunk
     static constexpr int kPCol = 256;                  // P_b at kPCol + 64 b
-    static constexpr int kOCol = 384;                  // O of item parity i at kOCol + 64 i
+    static constexpr int kOCol = 384;                  // O accumulator j at kOCol + D j
     static constexpr int kQ = 0;
     static constexpr int kK = kQ + QB * kQBytes;
     static constexpr int kV = kK + NST * kCBytes;
@@ -77,7 +86,8 @@ struct STCfg {
     static constexpr int kStats = kICnt + 16;                             // [item parity][half][row]: max, sum
     static constexpr int kXch = kStats + 2 * 2 * 128 * 8;                 // [chunk parity][half][row]: partial maxima
     static constexpr int kBars = kXch + 2 * 2 * 128 * 4;
-    static constexpr int bQFull = 0, bQEmpty = bQFull + QB, bKVFull = bQEmpty + QB, bKVEmpty = bKVFull + NST,
+    static constexpr int bQFull = 0, bQEmpty = bQFull + QB, bKFull = bQEmpty + QB, bVFull = bKFull + NST,
+                         bKVEmpty = bVFull + NST,
                          bListFull = bKVEmpty + NST, bListEmpty = bListFull + 2,
                          bSFull = bListEmpty + 2,
                          bPFull = bSFull + 2, bOReady = bPFull + 2, bOFree = bOReady + 2,
@@ -89,7 +99,7 @@ struct STCfg {
     static_assert(kBars % 8 == 0, "mbarriers need 8-byte alignment");
     static_assert(kStage % 16 == 0 && kStats % 8 == 0, "alignment of the stage and the stats");
     static_assert(kBytes + 1024 <= 232448, "shared memory budget");
-    static_assert(kOCol + 2 * D <= 512, "TMEM budget");
+    static_assert(kOCol + OB * D <= 512, "TMEM budget");
 };
 
 // One 128-query tile. LEVEL: tile `tile` of sorted block blk of problem prob = (bhi, node); CAUSAL: query tile gt of
@@ -157,10 +167,9 @@ __device__ __forceinline__ float exp_half(const uint32_t (&v)[64], float off, ui
     return l2.x + l2.y;
 }
 
-template <int MODE>
+template <int D, int MODE>
 __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) {
-    using C = STCfg;
-    constexpr int D = C::D;
+    using C = STCfg<D>;
     extern __shared__ unsigned char smem_raw[];
     const uint32_t raw_addr = smem_addr(smem_raw);
     const uint32_t pad = (1024u - (raw_addr & 1023u)) & 1023u;
@@ -179,7 +188,8 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
             mbar_init(bar(C::bQEmpty + i), 1);     // commit after the tile's last score product
         }
         for (int s = 0; s < C::NST; ++s) {
-            mbar_init(bar(C::bKVFull + s), 64);    // the K and V loader warps' lanes (copy completion)
+            mbar_init(bar(C::bKFull + s), 32);     // the K loader's lanes (copy completion)
+            mbar_init(bar(C::bVFull + s), 32);     // the V loader's lanes
             mbar_init(bar(C::bKVEmpty + s), 1);    // commit after the chunk's P.V product
         }
         for (int i = 0; i < 2; ++i) {
@@ -246,7 +256,9 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
             for (int64_t it = first; it < last && ok; it += stride, ++ni) {
                 const Tile x = decode_tile<MODE>(a, it);
                 const int ls = static_cast<int>(ni & 1);
-                if (ni >= 2 && !mbar_wait_inl(bar(C::bListEmpty + ls), ((ni >> 1) - 1) & 1, abort_flag)) {
+                // CAUSAL and DENSE read contiguous key rows: no list
+                if (is_level(MODE) && ni >= 2 &&
+                    !mbar_wait_inl(bar(C::bListEmpty + ls), ((ni >> 1) - 1) & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
@@ -287,25 +299,27 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
                         __syncwarp();
                     }
                 }
-                // LEVEL: chunks [0, ns) are sample chunks (their tails, past the block's count, point at the first
-                // key row and are masked), [ns, ns + nb) block chunks
-                for (int c = 0; c < x.nc; ++c) {
-                    const bool sample = is_level(MODE) && c < a.ns;
-                    const int u0 = c * kCK;
-                    const int64_t cbase = is_level(MODE) ? kbase : x.leaf_start + static_cast<int64_t>(c) * kCK;
+                if (is_level(MODE)) {
+                    // LEVEL: chunks [0, ns) are sample chunks (their tails, past the block's count, point at the first
+                    // key row and are masked), [ns, ns + nb) block chunks
+                    for (int c = 0; c < x.nc; ++c) {
+                        const bool sample = is_level(MODE) && c < a.ns;
+                        const int u0 = c * kCK;
+                        const int64_t cbase = is_level(MODE) ? kbase : x.leaf_start + static_cast<int64_t>(c) * kCK;
 #pragma unroll
-                    for (int rr = 0; rr < kCK / 32; ++rr) {
-                        const int row = rr * 32 + lane;
-                        int32_t loc;
-                        if (!is_level(MODE)) loc = row;
-                        else if (sample) loc = row + u0 < cnt ? slist[u0 + row] : 0;
-                        else loc = kperm[(c - a.ns) * kCK + row];
-                        ilist[c * kCK + row] = static_cast<int32_t>(cbase + loc);
+                        for (int rr = 0; rr < kCK / 32; ++rr) {
+                            const int row = rr * 32 + lane;
+                            int32_t loc;
+                            if (!is_level(MODE)) loc = row;
+                            else if (sample) loc = row + u0 < cnt ? slist[u0 + row] : 0;
+                            else loc = kperm[(c - a.ns) * kCK + row];
+                            ilist[c * kCK + row] = static_cast<int32_t>(cbase + loc);
+                        }
                     }
+                    if (lane == 0) icnt[ls] = is_level(MODE) ? cnt : 0;
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(C::bListFull + ls));
                 }
-                if (lane == 0) icnt[ls] = is_level(MODE) ? cnt : 0;
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(C::bListFull + ls));
                 // the query tile
                 const int qb = static_cast<int>(ni % C::QB), use = static_cast<int>(ni / C::QB);
                 if (use > 0 && !mbar_wait_inl(bar(C::bQEmpty + qb), (use - 1) & 1, abort_flag)) {
@@ -342,21 +356,40 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
             for (int64_t it = first; it < last && ok; it += stride, ++ni) {
                 const Tile x = decode_tile<MODE>(a, it);
                 const int ls = static_cast<int>(ni & 1);
-                if (!mbar_wait_inl(bar(C::bListFull + ls), (ni >> 1) & 1, abort_flag)) { ok = false; break; }
+                if (is_level(MODE) && !mbar_wait_inl(bar(C::bListFull + ls), (ni >> 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
                 const int32_t *ilist = reinterpret_cast<const int32_t *>(sm + C::kIList) + ls * (kMaxItemChunks * kCK);
                 for (int c = 0; c < x.nc; ++c, ++g) {
                     const int slot = static_cast<int>(g % C::NST);
                     const uint32_t round = g / C::NST;
-                    if (round > 0 && !mbar_wait_inl(bar(C::bKVEmpty + slot), (round - 1) & 1, abort_flag)) {
+                    // a stage is free once its previous chunk's products have read it. With two stages the K rows
+                    // are free as soon as that chunk's score product has completed (its commit to S_((g-2) mod 2)),
+                    // which lets K run a chunk ahead of the P.V products; otherwise both wait for the P.V product.
+                    bool free_ok = true;
+                    if (round > 0) {
+                        if (is_k && C::NST == 2) {
+                            const uint32_t gp = g - 2;
+                            free_ok = mbar_wait_inl(bar(C::bSFull + (gp & 1)), (gp >> 1) & 1, abort_flag);
+                        } else {
+                            free_ok = mbar_wait_inl(bar(C::bKVEmpty + slot), (round - 1) & 1, abort_flag);
+                        }
+                    }
+                    if (!free_ok) {
                         ok = false;
                         break;
                     }
-                    gather_rows<D, true, kCK>(dst0 + slot * C::kCBytes, src, 0, ilist + c * kCK, lane);
-                    cp_async_arrive(bar(C::bKVFull + slot));
+                    if (is_level(MODE))
+                        gather_rows<D, true, kCK>(dst0 + slot * C::kCBytes, src, 0, ilist + c * kCK, lane);
+                    else
+                        gather_rows<D, false, kCK>(dst0 + slot * C::kCBytes, src,
+                                                   x.leaf_start + static_cast<int64_t>(c) * kCK, ilist, lane);
+                    cp_async_arrive(bar((is_k ? C::bKFull : C::bVFull) + slot));
                 }
                 // the row indices are in registers once the copies are issued: the list slot may be rebuilt
                 __syncwarp();
-                if (ok && lane == 0) mbar_arrive(bar(C::bListEmpty + ls));
+                if (is_level(MODE) && ok && lane == 0) mbar_arrive(bar(C::bListEmpty + ls));
             }
             cp_wait<0>();
             if (!ok) flag_status(a.status);
@@ -383,14 +416,15 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
                     ++qc;
                 }
                 const int slot = static_cast<int>(ks % C::NST);
-                if (!mbar_wait_inl(bar(C::bKVFull + slot), (ks / C::NST) & 1, abort_flag)) return false;
+                if (!mbar_wait_inl(bar(C::bKFull + slot), (ks / C::NST) & 1, abort_flag)) return false;
                 tc_fence_after();
                 const int b = static_cast<int>(ks & 1);
                 const uint64_t dq = dq0 + static_cast<uint64_t>((qb_s * C::kQBytes) >> 4);
                 const uint64_t dk = dk0 + static_cast<uint64_t>((slot * C::kCBytes) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint64_t off = static_cast<uint64_t>((kk * 32) >> 4);
+                    // k-step kk: 16 columns inside 64-column slab kk / 4 (slabs of 128 rows x 128 bytes)
+                    const uint64_t off = static_cast<uint64_t>(((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4);
                     mma_ss(tmem + kCK * b, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(bar(C::bSFull + b));
@@ -407,25 +441,30 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
             uint32_t k = 0, ni = 0;
             for (int64_t it = first; it < last && ok; it += stride, ++ni) {
                 const Tile x = decode_tile<MODE>(a, it);
-                const int ip = static_cast<int>(ni & 1);
+                const int ob = static_cast<int>(ni % C::OB);
+                const uint32_t ouse = ni / C::OB;
                 for (int c = 0; c < x.nc && ok; ++c, ++k) {
                     const int b = static_cast<int>(k & 1);
                     const int slot = static_cast<int>(k % C::NST);
                     if (!mbar_wait_inl(bar(C::bPFull + b), (k >> 1) & 1, abort_flag)) { ok = false; break; }
-                    // the item's first P.V product overwrites the accumulator of parity ip: the epilogue must have read
-                    // item ni - 2's
-                    if (c == 0 && ni >= 2 && !mbar_wait_inl(bar(C::bOFree + ip), ((ni >> 1) - 1) & 1, abort_flag)) {
+                    // the item's first P.V product overwrites accumulator ob: the epilogue must have read the previous
+                    // item that used it (item ni - OB)
+                    if (c == 0 && ouse > 0 && !mbar_wait_inl(bar(C::bOFree + ob), (ouse - 1) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    if (!mbar_wait_inl(bar(C::bVFull + slot), (k / C::NST) & 1, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint64_t dv = dv0 + static_cast<uint64_t>((slot * C::kCBytes) >> 4);
-                    const uint32_t od = tmem + C::kOCol + D * ip;
+                    const uint32_t od = tmem + C::kOCol + D * ob;
 #pragma unroll
                     for (int kk = 0; kk < kCK / 16; ++kk)
                         mma_ts(od, tmem + C::kPCol + 64 * b + kk * 8, dv + static_cast<uint64_t>((kk * 2048) >> 4),
                                idesc_pv, (c > 0 || kk > 0) ? 1u : 0u);
-                    if (c == x.nc - 1) mma_commit(bar(C::bOReady + ip));
+                    if (c == x.nc - 1) mma_commit(bar(C::bOReady + ob));
                     mma_commit(bar(C::bKVEmpty + slot));   // both products of chunk k have been issued
                     ok = issue_next_s();                   // chunk k + 2 into buffer k mod 2
                 }
@@ -449,7 +488,8 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
         for (int64_t it = first; it < last && ok; it += stride, ++ni) {
             const Tile x = decode_tile<MODE>(a, it);
             const int ip = static_cast<int>(ni & 1);
-            const uint32_t tO = trow + C::kOCol + D * ip + 32 * h;   // this half's share of the row's accumulator
+            // this half's share (D / 2 columns) of the row's accumulator
+            const uint32_t tO = trow + C::kOCol + D * static_cast<int>(ni % C::OB) + (D / 2) * h;
             float m_run = -INFINITY, l = 0.0f;       // running max (base 2, weight included) and this half's sum
             // the item's count of kept samples (the valid columns of its sample chunks), from its list slot
             int cnt = 0;
@@ -518,17 +558,20 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
                 tmem_st32(trow + C::kPCol + 64 * b + 32 * h, pk);
                 if (rescale) {
                     // O holds the P.V products of the item's chunks before this one: wait for the last (chunk k - 1;
-                    // the commit that frees its K/V stage follows it), then scale this half's 32 of its columns
+                    // the commit that frees its K/V stage follows it), then scale this half's D / 2 of its columns
                     const uint32_t kp = k - 1;
                     if (!mbar_wait_inl(bar(C::bKVEmpty + kp % C::NST), (kp / C::NST) & 1, abort_flag)) ok = false;
                     if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
                     tc_fence_after();
-                    uint32_t o[32];
-                    tmem_ld32(tO, o);
-                    tmem_ld_wait();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                    tmem_st32(tO, o);
+                    for (int p32 = 0; p32 < D / 64; ++p32) {
+                        uint32_t o[32];
+                        tmem_ld32(tO + 32 * p32, o);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                        tmem_st32(tO + 32 * p32, o);
+                    }
                 }
                 tmem_st_wait();
                 tc_fence_before();
@@ -561,8 +604,9 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
                 const int64_t pos = static_cast<int64_t>(x.blk) * a.lv.bp + x.tile * 128 + r;
                 qloc = a.perm[(static_cast<int64_t>(x.prob) * 2) * a.lv.seg_len + pos];
             }
+            const int ob = static_cast<int>(ni % C::OB);
             if (!mbar_wait_inl(bar(C::bStatsReady + ip), par, abort_flag)) ok = false;
-            if (ok && !mbar_wait_inl(bar(C::bOReady + ip), par, abort_flag)) ok = false;
+            if (ok && !mbar_wait_inl(bar(C::bOReady + ob), (ni / C::OB) & 1, abort_flag)) ok = false;
             if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
             const float2 st0 = stats[(ip * 2) * 128 + r], st1 = stats[(ip * 2 + 1) * 128 + r];
             mbar_arrive(bar(C::bStatsFree + ip));
@@ -571,7 +615,7 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
             const float lsum = st0.y + st1.y;
             const float inv_l = 1.0f / lsum;
             const float Lrow = (st0.x + __log2f(lsum)) * kLn2;   // natural log of the row's normaliser
-            const uint32_t tOr = trow + C::kOCol + D * ip;
+            const uint32_t tOr = trow + C::kOCol + D * ob;
             // the row times `scale`: 16 columns [16 g, 16 g + 16) at a time
             auto merged16 = [&](int g, float scale, float (&vv)[16]) {
                 uint32_t o[16];
@@ -581,23 +625,31 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
                 for (int e = 0; e < 16; ++e) vv[e] = __uint_as_float(o[e]) * scale;
             };
             if (MODE != MODE_CAUSAL && !(is_level(MODE) && a.lv.level > 0) && a.out_dtype == 0) {
-                // bf16 output rows: the merged row packed into registers, the accumulators released, then the stores
-                uint4 seg[8];
-#pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    float vv[16];
-                    merged16(g, inv_l, vv);
-                    seg[2 * g] = make_uint4(pack_bf16x2(vv[0], vv[1]), pack_bf16x2(vv[2], vv[3]),
-                                            pack_bf16x2(vv[4], vv[5]), pack_bf16x2(vv[6], vv[7]));
-                    seg[2 * g + 1] = make_uint4(pack_bf16x2(vv[8], vv[9]), pack_bf16x2(vv[10], vv[11]),
-                                                pack_bf16x2(vv[12], vv[13]), pack_bf16x2(vv[14], vv[15]));
-                }
-                tc_fence_before();
-                mbar_arrive(bar(C::bOFree + ip));
+                // bf16 output rows, 64 columns (128 bytes, one store segment) at a time. d = 64: the merged row is
+                // packed into registers and the accumulator released before the store; d = 128: the accumulator is
+                // released after the second half has been read.
                 const int64_t orow = is_level(MODE) ? static_cast<int64_t>(x.bhi) * a.n + a.lv.q_off +
                                                           static_cast<int64_t>(x.node) * a.lv.node_len + qloc
                                                     : x.leaf_start + static_cast<int64_t>(x.gt) * 128 + r;
-                warp_store_segment<128>(stage, static_cast<unsigned char *>(a.O) + orow * D * 2, 0, seg, lane);
+                unsigned char *drow = static_cast<unsigned char *>(a.O) + orow * D * 2;
+#pragma unroll
+                for (int hs = 0; hs < D / 64; ++hs) {
+                    uint4 seg[8];
+#pragma unroll
+                    for (int g4 = 0; g4 < 4; ++g4) {
+                        float vv[16];
+                        merged16(4 * hs + g4, inv_l, vv);
+                        seg[2 * g4] = make_uint4(pack_bf16x2(vv[0], vv[1]), pack_bf16x2(vv[2], vv[3]),
+                                                 pack_bf16x2(vv[4], vv[5]), pack_bf16x2(vv[6], vv[7]));
+                        seg[2 * g4 + 1] = make_uint4(pack_bf16x2(vv[8], vv[9]), pack_bf16x2(vv[10], vv[11]),
+                                                     pack_bf16x2(vv[12], vv[13]), pack_bf16x2(vv[14], vv[15]));
+                    }
+                    if (hs == D / 64 - 1) {
+                        tc_fence_before();
+                        mbar_arrive(bar(C::bOFree + ob));
+                    }
+                    warp_store_segment<128>(stage, drow, 128 * hs, seg, lane);
+                }
                 if (is_level(MODE) && a.lse) a.lse[orow] = Lrow;
             } else if (MODE != MODE_CAUSAL) {
                 // fp32 rows (level 0) or parts (causal levels): 16 merged columns at a time through the stage
@@ -626,7 +678,7 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
                     warp_store_segment<64>(stage, drow, 64 * g, seg, lane);
                 }
                 tc_fence_before();
-                mbar_arrive(bar(C::bOFree + ip));
+                mbar_arrive(bar(C::bOFree + ob));
             } else {
                 // exact causal leaf part merged with the level parts of this row (log space): level l holds the row
                 // when it lies in the lower half of its node
@@ -691,7 +743,7 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
                     }
                 }
                 tc_fence_before();
-                mbar_arrive(bar(C::bOFree + ip));
+                mbar_arrive(bar(C::bOFree + ob));
             }
         }
         if (!ok) flag_status(a.status);
@@ -705,10 +757,10 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
     }
 }
 
-template <int MODE>
+template <int D, int MODE>
 int launch_st_t(TcArgs args, int sms, cudaStream_t st) {
-    const size_t smem = STCfg::kBytes + 1024;
-    auto kern = attn_st_kernel<MODE>;
+    const size_t smem = STCfg<D>::kBytes + 1024;
+    auto kern = attn_st_kernel<D, MODE>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
         return -1;
     // one item per query tile, chunks of kCK keys
@@ -736,7 +788,12 @@ int launch_st_t(TcArgs args, int sms, cudaStream_t st) {
 // of ha_attn_tc.cu).
 int launch_attn_pp(int d, const attn::TcArgs &args, int sms, cudaStream_t st) {
     if (args.stall_ns > 0) return -2;   // the timeout test hook lives in the kernel of ha_attn_tc.cu
-    if (d == 64 && args.mode == attn::MODE_LEVEL) return launch_st_t<attn::MODE_LEVEL>(args, sms, st);
+    // Level mode only: for the exact causal leaves and dense attention one query tile per item loads every key
+    // chunk once per tile, and the two-tile items of ha_attn_tc.cu measured faster (2.08 against 2.58 ms for the
+    // leaves of the causal prefill workload).
+    if (args.mode != attn::MODE_LEVEL) return -2;
+    if (d == 64) return launch_st_t<64, attn::MODE_LEVEL>(args, sms, st);
+    if (d == 128) return launch_st_t<128, attn::MODE_LEVEL>(args, sms, st);
     return -2;
 }
 

@@ -35,21 +35,27 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes per launch of a kernel class from an ncu capture, valid only while the source file it was
 # taken from is unchanged (sha256 of the file at capture time).
 TRAFFIC = {
-    # 4-head capture of the 32-head workload (the full one is too large for a multi-pass capture), scaled x8
-    # by the rows processed: attention 205.8 MB read + 42.9 MB written per 4-head launch; hash 134.2 + 6.2 MB.
+    # 4-head captures of the 32-head workloads (the full ones are too large for a multi-pass capture), scaled x8
+    # by the rows processed: attention (level kernel of ha_attn_pp.cu) 205.8 MB read + 46.3 MB written per 4-head
+    # launch at n = 131072, d = 64, and 111.2 + 14.3 MB at n = 32768, d = 128; hash 134.3 + 6.5 MB.
     ("attn", "long_bf16_n131072", "tc"): {
-        "file": "ha_attn_tc.cu",
-        "sha256": "6650df5df3dc9d8021e437523ad21193b7fced4b1f61325e8162791b32184d18",
-        "bytes": 8 * (205_804_288 + 42_924_800)},
-    # row-norm sampling (--sampling rownorm), 4-head capture scaled x8: 206.0 MB read + 44.6 MB written
+        "file": "ha_attn_pp.cu",
+        "sha256": "4fb00256336cb5978b70e7342f9bc16d5db9d68b32fa043e8bda0e15df6a6f14",
+        "bytes": 8 * (205_787_904 + 46_345_984)},
+    ("attn", "mid_bf16_n32768", "tc"): {
+        "file": "ha_attn_pp.cu",
+        "sha256": "4fb00256336cb5978b70e7342f9bc16d5db9d68b32fa043e8bda0e15df6a6f14",
+        "bytes": 8 * (111_216_640 + 14_281_216)},
+    # row-norm sampling (--sampling rownorm; kernel of ha_attn_tc.cu), 4-head capture scaled x8: 206.0 MB read +
+    # 44.6 MB written (taken before that file last changed, so it is not reported)
     ("attn", "long_bf16_n131072", "tc", "rownorm"): {
         "file": "ha_attn_tc.cu",
         "sha256": "6650df5df3dc9d8021e437523ad21193b7fced4b1f61325e8162791b32184d18",
         "bytes": 8 * (206_016_256 + 44_589_056)},
     ("hash", "long_bf16_n131072", "tc"): {
         "file": "ha_hash.cu",
-        "sha256": "4590cdf32028d354a14840822c657310cf7c55c4363a9d576b207e5aa9b08c08",
-        "bytes": 8 * (134_242_560 + 6_169_856)},
+        "sha256": "1a375171594e17545bd7d5900ce2a4c678af7fe092264fc5a71b71c3c81842b5",
+        "bytes": 8 * (134_257_152 + 6_460_160)},
 }
 
 

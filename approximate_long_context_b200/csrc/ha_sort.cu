@@ -9,7 +9,7 @@
 // (least significant digit first). A pass is three launches:
 //   count   -- per 2048-row chunk of a segment, a shared-memory histogram of the digit;
 //   scan    -- per segment, turn the chunk histograms into the first output position of every
-//              (chunk, digit) pair (digit-major, chunks in order);
+//              (chunk, digit) pair (digit-major, chunks in order), with 1024 / radix threads per digit;
 //   scatter -- per chunk, 8 warps each own a contiguous 256-row slice; a warp finds the rows of equal digit
 //              inside a 32-row step with one ballot per digit bit and keeps running per-digit counters, so
 //              rows leave in their original order within each digit. The chunk is ordered in shared memory
@@ -63,44 +63,62 @@ __global__ void __launch_bounds__(256) sort_count_kernel(Level lv, const uint16_
     for (int b = threadIdx.x; b < ps.radix; b += blockDim.x) h[b] = cnt[b];
 }
 
+// Per segment: the first output position of every (chunk, digit) pair, digit-major and chunks in order. The
+// 1024 threads split into G = 1024 / radix groups per digit; group g sums, then numbers, chunks
+// [g * cpg, (g + 1) * cpg), so the chunk counts of a digit are read by G threads at once.
 __global__ void __launch_bounds__(1024) sort_scan_kernel(int radix, int cps, int32_t *__restrict__ hist) {
+    __shared__ int part[1024];                    // [group][digit]: the group's sum, then its first position
     __shared__ int tot[1 << kMaxPassBits];
     const int64_t s = blockIdx.x;
     int32_t *h = hist + s * cps * radix;
-    // the chunk counts of a digit are read 16 at a time, so that the loads are in flight together
-    constexpr int U = 16;
-    for (int b = threadIdx.x; b < radix; b += blockDim.x) {
-        int run = 0;
-        for (int c0 = 0; c0 < cps; c0 += U) {
+    const int G = radix >= 1024 ? 1 : 1024 / radix;
+    const int cpg = (cps + G - 1) / G;
+    const int b = threadIdx.x % radix, g = threadIdx.x / radix;
+    const bool active = g < G;
+    const int c0 = g * cpg, c1 = min(cps, c0 + cpg);
+    constexpr int U = 16;   // loads in flight together
+    if (active) {
+        int sum = 0;
+        for (int c = c0; c < c1; c += U) {
             int t[U];
 #pragma unroll
-            for (int u = 0; u < U; ++u) t[u] = c0 + u < cps ? h[(c0 + u) * radix + b] : 0;
+            for (int u = 0; u < U; ++u) t[u] = c + u < c1 ? h[(c + u) * radix + b] : 0;
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
-                if (c0 + u < cps) h[(c0 + u) * radix + b] = run;
-                run += t[u];
-            }
+            for (int u = 0; u < U; ++u) sum += t[u];
+        }
+        part[g * radix + b] = sum;
+    }
+    __syncthreads();
+    if (threadIdx.x < radix) {   // exclusive over the groups of digit b; the digit's total
+        int run = 0;
+        for (int gg = 0; gg < G; ++gg) {
+            const int t = part[gg * radix + b];
+            part[gg * radix + b] = run;
+            run += t;
         }
         tot[b] = run;
     }
     __syncthreads();
     // inclusive scan of the digit totals (Hillis-Steele; radix <= blockDim, one digit per thread)
-    const int b = threadIdx.x;
+    const int tb = threadIdx.x;
     for (int off = 1; off < radix; off <<= 1) {
-        const int add = (b < radix && b >= off) ? tot[b - off] : 0;
+        const int add = (tb < radix && tb >= off) ? tot[tb - off] : 0;
         __syncthreads();
-        if (b < radix) tot[b] += add;
+        if (tb < radix) tot[tb] += add;
         __syncthreads();
     }
-    if (b < radix) {
-        const int base = b == 0 ? 0 : tot[b - 1];
-        for (int c0 = 0; c0 < cps; c0 += U) {
+    if (active) {
+        int run = (b == 0 ? 0 : tot[b - 1]) + part[g * radix + b];
+        for (int c = c0; c < c1; c += U) {
             int t[U];
 #pragma unroll
-            for (int u = 0; u < U; ++u) t[u] = c0 + u < cps ? h[(c0 + u) * radix + b] : 0;
+            for (int u = 0; u < U; ++u) t[u] = c + u < c1 ? h[(c + u) * radix + b] : 0;
 #pragma unroll
             for (int u = 0; u < U; ++u)
-                if (c0 + u < cps) h[(c0 + u) * radix + b] = t[u] + base;
+                if (c + u < c1) {
+                    h[(c + u) * radix + b] = run;
+                    run += t[u];
+                }
         }
     }
 }

@@ -7,6 +7,8 @@
 #include <string>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/hyper_attn.h"
 #include "ha_internal.h"
 
@@ -376,8 +378,12 @@ int run_forward(hyper_attn_t h, const void *Q, const void *K, const void *V, voi
 
     int launches = 0;
     int family = 0;
-    // profiling: take two events from the pool (grow on demand) and record the first one
-    auto prof_begin = [&]() -> long {
+    // every kernel class's enqueue sits in an NVTX range (a no-op unless a tracing tool is attached); with
+    // profiling on, two events from the pool (grown on demand) bracket it on the stream
+    static const char *const kRangeName[HA_KC_COUNT] = {"ha:hash", "ha:sort", "ha:attn", "ha:causal_base",
+                                                        "ha:draws"};
+    auto prof_begin = [&](int cls) -> long {
+        nvtxRangePushA(kRangeName[cls]);
         if (!h->profiling) return -1;
         while (h->ev_pool.size() < h->ev_used + 2) {
             cudaEvent_t e;
@@ -390,6 +396,7 @@ int run_forward(hyper_attn_t h, const void *Q, const void *K, const void *V, voi
         return static_cast<long>(i);
     };
     auto prof_end = [&](long i, int cls, int k) {
+        nvtxRangePop();
         if (i < 0) return;
         cudaEventRecord(h->ev_pool[i + 1], st);
         h->recs.push_back({cls, k > 0 ? k : 0, static_cast<size_t>(i), static_cast<size_t>(i + 1)});
@@ -412,7 +419,7 @@ int run_forward(hyper_attn_t h, const void *Q, const void *K, const void *V, voi
         const ha::RowNormGeom g = ha::rownorm_geometry(s.n, s.causal, s.levels, s.m, s.nodes_total);
         int32_t *rS = reinterpret_cast<int32_t *>(ws + lay.rn_S);
         float *rlw = reinterpret_cast<float *>(ws + lay.rn_lw);
-        ev = prof_begin();
+        ev = prof_begin(HA_KC_DRAWS);
         kl = ha::launch_rownorm_draws(g, V, dtype, s.d, s.bh, seed, bh_offset, reinterpret_cast<float *>(ws + lay.rn_nrm),
                                       reinterpret_cast<double *>(ws + lay.rn_csum),
                                       reinterpret_cast<double *>(ws + lay.rn_cdf), rS, rlw, st);
@@ -422,7 +429,7 @@ int run_forward(hyper_attn_t h, const void *Q, const void *K, const void *V, voi
         Srn = rS;
         lwrn = rlw;
     }
-    ev = prof_begin();
+    ev = prof_begin(HA_KC_HASH);
     kl = ha::launch_hash(Q, K, dtype, s.bh, s.n, s.d, h->hostP.data(), s.r, rank, near, st);
     prof_end(ev, HA_KC_HASH, kl);
     if ((rc = count(kl, "hash"))) return rc;
@@ -436,7 +443,7 @@ int run_forward(hyper_attn_t h, const void *Q, const void *K, const void *V, voi
         const ha::Level lv = make_level(s, l);
         int32_t *perm = reinterpret_cast<int32_t *>(ws + lay.perm[i]);
         int32_t *inv = reinterpret_cast<int32_t *>(ws + lay.inv[i]);
-        ev = prof_begin();
+        ev = prof_begin(HA_KC_SORT);
         if (npass == 1) {
             kl = ha::launch_sort_pass(lv, rank, passes[0], nullptr, hist, perm, inv, st);
         } else {
@@ -452,7 +459,7 @@ int run_forward(hyper_attn_t h, const void *Q, const void *K, const void *V, voi
         float *Op = s.causal ? Opart + static_cast<size_t>(l - 1) * half_rows * s.d : nullptr;
         float *Lp = s.causal ? Lpart + static_cast<size_t>(l - 1) * half_rows : nullptr;
         int k = -2;
-        ev = prof_begin();
+        ev = prof_begin(HA_KC_ATTN);
         if (use_tc) family = HA_KERNEL_TC;
         if (use_tc)
             k = ha::launch_attn_tc(lv, Q, K, V, s.d, perm, inv, S, s.m, s.nodes_total, O, out_dtype, lse, Op, Lp,
@@ -466,7 +473,7 @@ int run_forward(hyper_attn_t h, const void *Q, const void *K, const void *V, voi
     }
     if (s.causal && !sort_only) {
         int k = -2;
-        ev = prof_begin();
+        ev = prof_begin(HA_KC_CAUSAL_BASE);
         if (use_tc && family != HA_KERNEL_SIMT) family = HA_KERNEL_TC;
         // a backward pass needs each row's final log normaliser, which the SIMT kernel writes
         if (use_tc && !h->bwd)

@@ -227,7 +227,10 @@ typedef enum {
 } ha_kernel_class;
 
 /* enable = 1: record a CUDA event pair on the handle's stream around every kernel class launch of the
- * following forward calls; 0: stop recording. Recording adds two event records per launch. */
+ * following forward calls; 0: stop recording. Recording adds two event records per launch.
+ * Independently of this switch, the host-side enqueue of every kernel class sits in an NVTX range named
+ * "ha:hash", "ha:sort", "ha:attn", "ha:causal_base" or "ha:draws", which tracing tools (Nsight Systems) show
+ * next to the kernels; without such a tool attached the ranges cost a few nanoseconds. */
 HA_API int hyper_attn_profile(hyper_attn_t h, int enable);
 
 /* Synchronise the handle's stream and add, per kernel class (array index = ha_kernel_class, n entries),

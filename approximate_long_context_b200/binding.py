@@ -11,7 +11,11 @@ import os
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
+# HA_LIBRARY=debug selects the HA_DEBUG build (bounds-checked index reads), any other value a library path
 LIB_PATH = os.path.join(_HERE, "libhyper_attn.so")
+if os.environ.get("HA_LIBRARY"):
+    LIB_PATH = (os.path.join(_HERE, "libhyper_attn_debug.so") if os.environ["HA_LIBRARY"] == "debug"
+                else os.environ["HA_LIBRARY"])
 
 HA_OK, HA_ERR_INVALID_ARG, HA_ERR_UNSUPPORTED, HA_ERR_CUDA, HA_ERR_OOM, HA_ERR_TIMEOUT = 0, -1, -2, -3, -4, -5
 DTYPES = {"bf16": 0, "fp32": 1}

@@ -866,6 +866,9 @@ int hyper_attn_status(hyper_attn_t h) {
     if (word) {
         HA_CUDA(h, cudaMemset(h->ws + h->lay.status, 0, sizeof word));
         if (word & ha::kStatusTimeout) return fail(h, HA_ERR_TIMEOUT, "a device-side wait gave up (status %d)", word);
+        if (word & ha::kStatusBounds)
+            return fail(h, HA_ERR_CUDA, "a row index read from a permutation or a sample list was out of range, "
+                                        "HA_DEBUG build (status %d)", word);
         return fail(h, HA_ERR_CUDA, "device status word %d", word);
     }
     return HA_OK;

@@ -133,6 +133,35 @@ __device__ __forceinline__ void flag_status(int *status) {
     if (status) atomicOr(status, kStatusTimeout);
 }
 
+// HA_DEBUG builds: a row index read from data (a permutation, a sample list) outside [0, limit) sets
+// kStatusBounds in the status word and is replaced by 0, so that the kernel reads a valid row instead of
+// faulting. Regular builds compile the check away.
+__device__ __forceinline__ int32_t checked_index(int32_t i, int64_t limit, int *status) {
+#ifdef HA_DEBUG
+    if (i < 0 || i >= limit) {
+        if (status) atomicOr(status, kStatusBounds);
+        return 0;
+    }
+#endif
+    (void)limit;
+    (void)status;
+    return i;
+}
+
+// The same check, in place, on `count` entries of an index array in shared memory (the warp's lanes strided).
+__device__ __forceinline__ void check_indices(int32_t *idx, int count, int64_t limit, int *status, int lane) {
+#ifdef HA_DEBUG
+    __syncwarp();
+    for (int i = lane; i < count; i += 32) idx[i] = checked_index(idx[i], limit, status);
+    __syncwarp();
+#endif
+    (void)idx;
+    (void)count;
+    (void)limit;
+    (void)status;
+    (void)lane;
+}
+
 // One SEG-byte segment, at byte offset `off`, of each of the warp's 32 output rows: lane l holds the segment of
 // its own row (16-byte pieces pc[0..SEG/16)) and `drow` points at the start of that row. The segments pass
 // through the warp's shared-memory stage (32 x SEG bytes, pieces XOR-swizzled so that neither the row-wise

@@ -273,6 +273,7 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
                         __syncwarp();
                         for (int i = lane; i < a.lv.bp / 4; i += 32)
                             reinterpret_cast<int4 *>(kperm)[i] = reinterpret_cast<const int4 *>(pkg)[i];
+                        check_indices(kperm, a.lv.bp, a.lv.seg_len, a.status, lane);
                         cnt = 0;
                         if (a.m > 0) {
                             if (static_cast<int64_t>(x.prob) != cached_prob) {
@@ -280,7 +281,8 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
                                     a.S + (static_cast<int64_t>(x.bhi) * a.nodes_total + (a.lv.heap0 + x.node - 1)) * a.m;
                                 const int32_t *ik = a.inv + (static_cast<int64_t>(x.prob) * 2 + 1) * a.lv.seg_len;
                                 __syncwarp();
-                                for (int u = lane; u < a.m; u += 32) cache_s[u] = Sp[u];
+                                for (int u = lane; u < a.m; u += 32)
+                                    cache_s[u] = checked_index(Sp[u], a.lv.seg_len, a.status);
                                 __syncwarp();
                                 for (int u = lane; u < a.m; u += 32) cache_b[u] = ik[cache_s[u]] / a.lv.bp;
                                 cached_prob = x.prob;
@@ -332,6 +334,7 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
                                         static_cast<int64_t>(x.blk) * a.lv.bp + x.tile * 128;
                     __syncwarp();
                     reinterpret_cast<int4 *>(qperm)[lane] = reinterpret_cast<const int4 *>(pq)[lane];
+                    check_indices(qperm, 128, a.lv.seg_len, a.status, lane);
                     __syncwarp();
                     gather_rows<D, true>(base, a.Q,
                                          static_cast<int64_t>(x.bhi) * a.n + static_cast<int64_t>(x.node) * a.lv.node_len +
@@ -602,7 +605,8 @@ __global__ void __launch_bounds__(kSTThreads, 1) attn_st_kernel(const TcArgs a) 
             int64_t qloc = 0;
             if (is_level(MODE)) {
                 const int64_t pos = static_cast<int64_t>(x.blk) * a.lv.bp + x.tile * 128 + r;
-                qloc = a.perm[(static_cast<int64_t>(x.prob) * 2) * a.lv.seg_len + pos];
+                qloc = checked_index(a.perm[(static_cast<int64_t>(x.prob) * 2) * a.lv.seg_len + pos], a.lv.seg_len,
+                                     a.status);
             }
             const int ob = static_cast<int>(ni % C::OB);
             if (!mbar_wait_inl(bar(C::bStatsReady + ip), par, abort_flag)) ok = false;

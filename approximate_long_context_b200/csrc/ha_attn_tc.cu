@@ -206,6 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
             const int32_t *pq = a.perm + (x.prob * 2) * a.lv.seg_len + x.blk * a.lv.bp + (x.pair * 2 + t) * 128;
             __syncwarp();
             reinterpret_cast<int4 *>(qperm)[lane] = reinterpret_cast<const int4 *>(pq)[lane];
+            check_indices(qperm, 128, a.lv.seg_len, a.status, lane);
             __syncwarp();
             qbase = x.bhi * a.n + x.node * a.lv.node_len + a.lv.q_off;
         } else {
@@ -254,19 +255,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                 __syncwarp();
                 for (int i = lane; i < a.lv.bp / 4; i += 32)
                     reinterpret_cast<int4 *>(kperm)[i] = reinterpret_cast<const int4 *>(pkg)[i];
+                check_indices(kperm, a.lv.bp, a.lv.seg_len, a.status, lane);
                 if (a.ns > 0) {
                     if (x.prob != cached_prob) {
                         const int32_t *Sp = a.S + (x.bhi * a.nodes_total + (a.lv.heap0 + x.node - 1)) * a.m;
                         const int32_t *ik = a.inv + (x.prob * 2 + 1) * a.lv.seg_len;
                         __syncwarp();
-                        for (int u = lane; u < a.m; u += 32) cache_s[u] = Sp[u];
+                        for (int u = lane; u < a.m; u += 32)
+                            cache_s[u] = checked_index(Sp[u], a.lv.seg_len, a.status);
                         __syncwarp();
                         for (int u = lane; u < a.m; u += 32) cache_b[u] = ik[cache_s[u]] / a.lv.bp;
                         if (MODE == MODE_LEVEL_RN) {
                             // row-norm draws of this problem behind the uniform samples; -1 (no draw) never kept
                             const int64_t so = (x.bhi * a.nodes_total + (a.lv.heap0 + x.node - 1)) * a.m;
                             for (int u = lane; u < a.m; u += 32) {
-                                cache_s[a.m + u] = a.Srn[so + u];
+                                const int32_t sr = a.Srn[so + u];   // -1: no draw
+                                cache_s[a.m + u] = sr < 0 ? sr : checked_index(sr, a.lv.seg_len, a.status);
                                 cache_w[u] = a.lwrn[so + u] * kLog2e;
                             }
                             __syncwarp();
@@ -563,7 +567,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
             int64_t qloc = 0;
             if (is_level(MODE)) {
                 const int64_t pos = x.blk * a.lv.bp + (x.pair * 2 + t) * 128 + r;
-                qloc = a.perm[(x.prob * 2) * a.lv.seg_len + pos];   // consumed by the epilogue
+                // consumed by the epilogue
+                qloc = checked_index(a.perm[(x.prob * 2) * a.lv.seg_len + pos], a.lv.seg_len, a.status);
             }
             float m_run = -INFINITY, l = 0.0f;
             for (int c = 0; c < my_nc; ++c) {

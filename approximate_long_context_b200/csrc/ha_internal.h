@@ -13,6 +13,7 @@ constexpr int kSortWarps = 8;
 
 // Device status word bits (written by kernels that wait with a bound, read by hyper_attn_status).
 constexpr int kStatusTimeout = 1;
+constexpr int kStatusBounds = 2;     // HA_DEBUG builds: a row index read from data was out of range
 
 // One level of the computation. Level 0 is the non-causal problem (one node covering all n rows);
 // causal level l >= 1 has nodes of node_len = n >> (l-1) rows whose off-diagonal problem pairs the

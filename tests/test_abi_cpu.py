@@ -40,6 +40,15 @@ def test_exports_every_declared_symbol(lib):
     assert set(names) <= set(binding.EXPORTS)
 
 
+def test_debug_build_exports_every_declared_symbol(lib):
+    """The HA_DEBUG build (bounds-checked index reads in the tensor-core kernels) is the same library."""
+    from approximate_long_context_b200 import build
+    path = build.build(debug=True)
+    dbg = ctypes.CDLL(path)
+    for name in declared_functions():
+        assert hasattr(dbg, name), name
+
+
 def test_version(lib):
     assert lib.hyper_attn_version() >= 100
 

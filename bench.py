@@ -36,16 +36,16 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # taken from is unchanged (sha256 of the file at capture time).
 TRAFFIC = {
     # 4-head captures of the 32-head workloads (the full ones are too large for a multi-pass capture), scaled x8
-    # by the rows processed: attention (level kernel of ha_attn_pp.cu) 205.8 MB read + 46.3 MB written per 4-head
-    # launch at n = 131072, d = 64, and 111.2 + 14.3 MB at n = 32768, d = 128; hash 134.3 + 6.5 MB.
+    # by the rows processed: attention (level kernel of ha_attn_pp.cu) 205.8 MB read + 46.5 MB written per 4-head
+    # launch at n = 131072, d = 64, and 111.2 + 15.8 MB at n = 32768, d = 128; hash 134.3 + 6.5 MB.
     ("attn", "long_bf16_n131072", "tc"): {
         "file": "ha_attn_pp.cu",
-        "sha256": "4fb00256336cb5978b70e7342f9bc16d5db9d68b32fa043e8bda0e15df6a6f14",
-        "bytes": 8 * (205_787_904 + 46_345_984)},
+        "sha256": "136d222295ffc01aedb9edce94d2b595377c094757c4b9293213988f423f0523",
+        "bytes": 8 * (205_786_880 + 46_522_880)},
     ("attn", "mid_bf16_n32768", "tc"): {
         "file": "ha_attn_pp.cu",
-        "sha256": "4fb00256336cb5978b70e7342f9bc16d5db9d68b32fa043e8bda0e15df6a6f14",
-        "bytes": 8 * (111_216_640 + 14_281_216)},
+        "sha256": "136d222295ffc01aedb9edce94d2b595377c094757c4b9293213988f423f0523",
+        "bytes": 8 * (111_241_728 + 15_828_736)},
     # row-norm sampling (--sampling rownorm; kernel of ha_attn_tc.cu), 4-head capture scaled x8: 206.0 MB read +
     # 44.6 MB written (taken before that file last changed, so it is not reported)
     ("attn", "long_bf16_n131072", "tc", "rownorm"): {

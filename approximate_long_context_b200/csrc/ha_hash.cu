@@ -13,10 +13,10 @@
 // g = ((bh*2 + which)*n + row) (which 0 = Q, 1 = K), RPT rows per thread. Tiles are double-buffered in
 // shared memory: the 16-byte cp.async copies of tile i+1 (coalesced; row stride padded by 16 bytes against
 // bank conflicts) are in flight while tile i is hashed. P travels as a kernel parameter ([d][r4], r rounded
-// up to a multiple of 4). d = 64: the loops over k and j are unrolled, so every fused multiply-add takes its
-// P[k][j] straight from the constant bank, with no load instruction. d = 128: that unrolled body (twice the size)
-// no longer fits the instruction cache, so P is copied to shared memory and each broadcast 16-byte load of it
-// feeds both of a thread's rows.
+// up to a multiple of 4): the loops over k and j are unrolled, so every fused multiply-add takes its P[k][j]
+// straight from the constant bank, with no load instruction. A thread hashes two rows for d = 64 and one for
+// d = 128, so that the unrolled body has the same size for both (with two rows at d = 128 it outgrew the
+// instruction cache).
 #include "ha_common.cuh"
 #include "ha_internal.h"
 
@@ -45,15 +45,10 @@ __global__ void __launch_bounds__(kThreads) hash_kernel(const void *__restrict__
     constexpr int EPC = 16 / ESZ;          // elements per 16-byte chunk
     // R4: r rounded up to a multiple of 4 (compile time, so the unrolled loops carry no conditions); the
     // padded projections multiply zero columns of P and are ignored.
-    constexpr bool kConstP = D == 64;
-    constexpr int PS = R4 > 0 ? R4 : 4;
     extern __shared__ __align__(16) unsigned char smem[];
-    float *Ps = reinterpret_cast<float *>(smem);                               // [D][PS] (d = 128)
-    unsigned char *tiles = smem + (kConstP ? 0 : D * PS * sizeof(float));      // [2][kRows][STRIDE]
+    unsigned char *tiles = smem;                                               // [2][kRows][STRIDE]
 
     const int tid = threadIdx.x;
-    if (!kConstP)
-        for (int i = tid; i < D * PS; i += kThreads) Ps[i] = R4 > 0 ? P.v[i] : 0.0f;
     const int64_t ntiles = (total_rows + kRows - 1) / kRows;
 
     // stage one tile with 16-byte copies. A tile inside one segment (the usual case) is kRows * ROW_BYTES
@@ -96,7 +91,7 @@ __global__ void __launch_bounds__(kThreads) hash_kernel(const void *__restrict__
         } else {
             cp_async_wait<0>();
         }
-        __syncthreads();   // tile `buf` (and P on the first pass, d = 128) visible to every thread
+        __syncthreads();   // tile `buf` visible to every thread
 
         const unsigned char *rows = tiles + buf * (kRows * STRIDE) + tid * STRIDE;
         float acc[RPT][R4 > 0 ? R4 : 1];
@@ -107,7 +102,7 @@ __global__ void __launch_bounds__(kThreads) hash_kernel(const void *__restrict__
 #pragma unroll
             for (int j = 0; j < R4; ++j) acc[q][j] = 0.0f;
         }
-#pragma unroll(kConstP ? CHUNKS : 2)
+#pragma unroll
         for (int c = 0; c < CHUNKS; ++c) {
             float x[RPT][EPC];
 #pragma unroll
@@ -132,26 +127,11 @@ __global__ void __launch_bounds__(kThreads) hash_kernel(const void *__restrict__
                 const int k = c * EPC + e;
 #pragma unroll
                 for (int q = 0; q < RPT; ++q) nrm2[q] = __fmaf_rn(x[q][e], x[q][e], nrm2[q]);
-                if constexpr (kConstP) {
 #pragma unroll
-                    for (int j = 0; j < R4; ++j) {
-                        const float p = P.v[k * R4 + j];
+                for (int j = 0; j < R4; ++j) {
+                    const float p = P.v[k * R4 + j];
 #pragma unroll
-                        for (int q = 0; q < RPT; ++q) acc[q][j] = __fmaf_rn(x[q][e], p, acc[q][j]);
-                    }
-                } else {
-                    const float4 *pk = reinterpret_cast<const float4 *>(Ps + k * PS);
-#pragma unroll
-                    for (int q4 = 0; q4 < R4 / 4; ++q4) {
-                        const float4 p = pk[q4];
-#pragma unroll
-                        for (int q = 0; q < RPT; ++q) {
-                            acc[q][4 * q4 + 0] = __fmaf_rn(x[q][e], p.x, acc[q][4 * q4 + 0]);
-                            acc[q][4 * q4 + 1] = __fmaf_rn(x[q][e], p.y, acc[q][4 * q4 + 1]);
-                            acc[q][4 * q4 + 2] = __fmaf_rn(x[q][e], p.z, acc[q][4 * q4 + 2]);
-                            acc[q][4 * q4 + 3] = __fmaf_rn(x[q][e], p.w, acc[q][4 * q4 + 3]);
-                        }
-                    }
+                    for (int q = 0; q < RPT; ++q) acc[q][j] = __fmaf_rn(x[q][e], p, acc[q][j]);
                 }
             }
         }
@@ -195,10 +175,11 @@ int launch_hash_t(const void *Q, const void *K, int64_t bh, int64_t n, const flo
     for (int k = 0; k < D; ++k)
         for (int j = 0; j < r; ++j) proj.v[k * R4 + j] = P[k * r + j];
     constexpr int ESZ = DTYPE == 0 ? 2 : 4;
-    // two rows per thread while a double-buffered tile stays small (rows of up to 256 bytes)
-    constexpr int RPT = D * ESZ <= 256 ? 2 : 1;
+    // two rows per thread for d = 64, one for d = 128: the unrolled chain body (d x RPT x r fused multiply-adds)
+    // then has the same size for both and fits the instruction cache
+    constexpr int RPT = D == 64 ? 2 : 1;
     constexpr int kRows = kThreads * RPT;
-    const size_t smem = (D == 64 ? 0 : D * (R4 > 0 ? R4 : 4) * sizeof(float)) + 2 * kRows * (D * ESZ + 16);
+    const size_t smem = 2 * kRows * (D * ESZ + 16);
     auto kern = hash_kernel<D, DTYPE, R4, RPT>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
         return -1;

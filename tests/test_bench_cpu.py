@@ -49,3 +49,31 @@ def test_work_model():
     assert f == 0 and b == w.bh * 2 * w.n * (w.d * 2 + 3)
     assert bench.nlev_of(w) == 0
     assert bench.nlev_of(wl.WORKLOADS["prefill_causal_bf16_n32768"]) == 3
+
+
+def test_step_work_model():
+    """The whole-step work behind `roofline_step`: the headline step is HBM-bound (0.51 ms of bytes against
+    0.33 ms of flops at the measured peaks), and the causal model adds the exact leaves and the level parts."""
+    w = wl.WORKLOADS[wl.HEADLINE]
+    b, f = bench.step_work(w)
+    n, d, bh = w.n, w.d, w.bh
+    # hash reads Q, K; attention reads Q, K, V and writes O (2-byte elements); ranks and permutations 32 B per row
+    assert b == bh * (6.0 * n * d * 2 + 32.0 * n)
+    assert f == bh * 4.0 * n * d * (w.block + w.m)
+    assert f == bench.algorithmic(w, "attn")[1]
+    c = wl.WORKLOADS["prefill_causal_bf16_n32768"]
+    L = bench.nlev_of(c)
+    bc, fc = bench.step_work(c)
+    assert fc == c.bh * 2.0 * c.n * c.d * (c.base + L * (c.block + c.m))
+    assert bc == c.bh * ((6.0 * c.n * c.d + 1.5 * L * c.n * c.d) * 2 + 32.0 * c.n * (L + 1))
+    # fp32 inputs double the element bytes
+    t = wl.WORKLOADS["tiny_fp32_n1024"]
+    bt, _ = bench.step_work(t)
+    assert bt == t.bh * (6.0 * t.n * t.d * 4 + 32.0 * t.n)
+
+
+def test_traffic_entries_name_existing_sources():
+    """Every recorded ncu traffic figure names a source file of the library and a 64-hex-digit hash."""
+    for key, tr in bench.TRAFFIC.items():
+        assert os.path.exists(os.path.join(ROOT, "approximate_long_context_b200", "csrc", tr["file"])), key
+        assert len(tr["sha256"]) == 64 and tr["bytes"] > 0, key

@@ -722,17 +722,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const TcArgs a) {
                             pk[16 + 2 * e + 1] = pack_bf16x2(b2, b3);
                         }
                     } else {
+                        // scale-and-offset and sums as packed f32x2 instructions, the exponentials on the MUFU unit
+                        const uint64_t sc = f2_pack(kLog2e, kLog2e), of = f2_pack(off, off);
+                        uint64_t sa = f2_pack(0.0f, 0.0f), sb = sa;
 #pragma unroll
                         for (int e = 0; e < 16; ++e) {
-                            const float p0 = ex2_approx(fmaf(__uint_as_float(va[2 * e]), kLog2e, off));
-                            const float p1 = ex2_approx(fmaf(__uint_as_float(va[2 * e + 1]), kLog2e, off));
-                            const float p2 = ex2_approx(fmaf(__uint_as_float(vb[2 * e]), kLog2e, off));
-                            const float p3 = ex2_approx(fmaf(__uint_as_float(vb[2 * e + 1]), kLog2e, off));
-                            l0 += p0 + p1;
-                            l1 += p2 + p3;
+                            const float2 xa =
+                                f2_unpack(f2_fma(f2_pack(__uint_as_float(va[2 * e]), __uint_as_float(va[2 * e + 1])), sc, of));
+                            const float2 xb =
+                                f2_unpack(f2_fma(f2_pack(__uint_as_float(vb[2 * e]), __uint_as_float(vb[2 * e + 1])), sc, of));
+                            const float p0 = ex2_approx(xa.x), p1 = ex2_approx(xa.y);
+                            const float p2 = ex2_approx(xb.x), p3 = ex2_approx(xb.y);
+                            sa = f2_add(sa, f2_pack(p0, p1));
+                            sb = f2_add(sb, f2_pack(p2, p3));
                             pk[e] = pack_bf16x2(p0, p1);
                             pk[16 + e] = pack_bf16x2(p2, p3);
                         }
+                        const float2 ta = f2_unpack(sa), tb = f2_unpack(sb);
+                        l0 += ta.x + ta.y;
+                        l1 += tb.x + tb.y;
                     }
                     if (to_o) tmem_st32(tP + h * 32, pk);
                 }

@@ -517,6 +517,8 @@ def run_ours(args, w: wl.Workload):
             "config": config_of(w, args.sampling),
             "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                          "frac": achieved / peak, "traffic": traffic, "kernel": dom,
+                         # against the bf16 peak sustained for seconds under the power cap (context)
+                         "frac_sustained": (achieved / peaks["bf16_tflops_sustained"]) if bound == "tensor" else None,
                          "kernel_ms_per_launch": avg_ms, "peak_source": peak_src + (" burst" if bound == "tensor" else ""),
                          "kernel_family": "tcgen05" if family == "tc" else "simt"},
             "roofline_step": roof_step,

@@ -114,3 +114,18 @@ def test_default_options_match_the_binding_defaults(lib):
     lib.hyper_attn_default_options(ctypes.byref(o))
     assert (o.dtype, o.out_dtype, o.batch, o.causal_base, o.kernel, o.debug_captures, o.bh_offset,
             o.test_stall_ms, o.sampling) == (0, -1, 1, 4096, 0, 0, 0, 0, 0)
+
+
+def test_binding_selects_the_debug_build():
+    """HA_LIBRARY=debug makes the binding load the HA_DEBUG build (in a fresh process); unset, the regular one."""
+    import subprocess
+    import sys
+    code = "from approximate_long_context_b200 import binding; print(binding.LIB_PATH)"
+    env = dict(os.environ, HA_LIBRARY="debug")
+    out = subprocess.run([sys.executable, "-c", code], env=env, cwd=ROOT, capture_output=True, text=True,
+                         check=True).stdout.strip()
+    assert out.endswith("libhyper_attn_debug.so")
+    env.pop("HA_LIBRARY")
+    out = subprocess.run([sys.executable, "-c", code], env=env, cwd=ROOT, capture_output=True, text=True,
+                         check=True).stdout.strip()
+    assert out.endswith("libhyper_attn.so")

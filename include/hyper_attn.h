@@ -213,7 +213,9 @@ typedef enum {
 HA_API int hyper_attn_debug_copy(hyper_attn_t h, int what, int level, void *host_dst, size_t bytes);
 
 /* Synchronise the handle's stream and report device-side status: HA_OK, HA_ERR_TIMEOUT if a bounded
- * wait gave up, or HA_ERR_CUDA if the stream holds an error. Clears the device status word. */
+ * wait gave up, or HA_ERR_CUDA if the stream holds an error or (HA_DEBUG build, libhyper_attn_debug.so) a
+ * tensor-core kernel read a row index out of range from a permutation or a sample list (it then read row 0
+ * instead). Clears the device status word. */
 HA_API int hyper_attn_status(hyper_attn_t h);
 
 /* Kernel classes for profiling. */
